@@ -1,0 +1,89 @@
+// Batched square GEMM on split-fp16 operands with a fused epilogue.
+//
+// Every product on the hot path of the batched block-Shampoo step is a
+// B x B x B product of two matrices from stacked (N, B, B) tensors (the DASH
+// explainer's "Building blocks": stack blocks into (N, B, B), run batched
+// products).  Operands are held as two fp16 planes (hi, lo * 2^11) and the
+// kernel accumulates hi*hi and hi*lo + lo*hi in two fp32 tensor-memory
+// accumulators (tcgen05, kind::f16), which gives about fp32 accuracy at the
+// fp16 tensor-core rate.
+//
+// Both operands are read K-major: problem p computes
+//     out_p = s_p * (alpha * A_p Bm_p^T + beta * Cin_p + gamma * I)
+// where A_p and Bm_p are row-major matrices of the operand stacks.  A product
+// A * B is therefore formed from a stored B^T (the library keeps transposed
+// copies where an iterate is not symmetric).  A launch carries one or two
+// "ops" (groups of problems) with their own operand stacks and epilogues.
+// With sym = 1 only upper-triangle tiles are computed and each off-diagonal
+// tile is also written mirrored (for results that are symmetric by
+// construction).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace dash {
+
+// One Shampoo block in parameter layout (used by the preconditioner epilogue
+// that scatters U into the parameter-shaped buffer).
+struct BlockDesc {
+  long long off;  // element offset of the owning parameter in the flat buffer
+  int pitch;      // row length (columns) of the owning parameter
+  int r0, c0;     // block origin inside the parameter
+  int br, bc;     // block extent (<= B)
+  int param;      // owning parameter index
+};
+
+// Matrix index of problem p: base + stride * (p % mod); mod <= 0 means no
+// modulo and stride 0 means 1, so a zero-initialised Idx maps p to p.
+struct Idx {
+  int base, mod, stride;
+};
+
+struct GemmOp {
+  int nprob;
+  Idx a, b;                  // operand matrices in this op's A / Bm stacks
+  float alpha, beta, gamma;
+  const float* scale;        // per-problem multiplier s_p (nullptr: 1)
+  Idx scale_i;
+  const __half* cin_split;   // split Cin stack (nullptr: none)
+  Idx cin_i;
+  int cin_trans;             // 1: Cin_p(r, c) is read from element (c, r)
+  const float* cin_f32;      // fp32 Cin stack (nullptr: none)
+  Idx cinf_i;
+  __half* out_split;         // split output, as computed (+ mirror if sym)
+  Idx out_i;
+  __half* outt_split;        // split output, transposed (non-sym only)
+  Idx outt_i;
+  float* out_f32;            // fp32 output, as computed (+ mirror if sym)
+  Idx outf_i;
+  float* outt_f32;           // fp32 output, transposed (non-sym only)
+  Idx outtf_i;
+  const BlockDesc* blocks;   // non-null: scatter out_p into u_out (parameter layout)
+  float* u_out;
+  float* unorm;              // per-problem sum of squares of the scattered out_p
+};
+
+struct GemmArgs {
+  int B;      // matrix size; multiple of 128
+  int sym;    // 1: symmetric outputs (upper-triangle tiles + mirrored writes)
+  int nops;   // 1 or 2
+  GemmOp op[2];
+  unsigned* status;  // device status word (non-finite / timeout bits)
+};
+
+// Operand stacks of one op: split stacks of B x B matrices, layout
+// [matrix][plane][row][col] fp16.
+struct OpBuffers {
+  const __half* a;
+  int a_nmat;
+  const __half* b;
+  int b_nmat;
+};
+
+// Launch one batched GEMM (args.nops ops).  Returns cudaSuccess or the
+// launch / encode error.
+cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaStream_t stream);
+
+}  // namespace dash

@@ -1,0 +1,78 @@
+// Memory-bound kernels of the batched block-Shampoo step: power iteration,
+// solver prologues, gradient gather, Adam graft and update.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "gemm.cuh"
+
+namespace dash {
+
+constexpr int kPiStarts = 32;  // power-iteration start vectors per factor
+
+// Per-parameter metadata used by the Adam / update kernels.
+struct ParamDev {
+  const float* grad;
+  float* param;
+  float* m;
+  float* v;
+  long long uoff;       // offset of this parameter in the flat U buffer
+  long long item_base;  // first work item (one item = 1024 columns of one row)
+  int rows, cols;
+  int blk_base;         // index of the parameter's first block
+  int ncb;              // column blocks
+  int chunks;           // 1024-column chunks per row
+  int vec;              // 1: float4 path (cols % 4 == 0, 16-byte aligned)
+};
+
+// Power iteration: one product W_next = (F + eps I) V on every factor, where
+// V = v0 (first product, t = 0) or W_prev with unit columns.  Rows/columns at
+// or beyond a factor's true size are treated as zero.  Accumulates per column
+// ||W_next||^2, V.W_next and V.V into stats_next ((nf, 3, 32), zeroed).
+void launch_pi_iter(const float* F, int nf, int B, float eps, const int* fsize, const float* v0,
+                    const float* W_prev, const float* stats_prev, float* W_next, float* stats_next,
+                    cudaStream_t st);
+
+// lambda[f] = max_j (V.W)_j / (V.V)_j from the last product's statistics.
+void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* lambda_out, cudaStream_t st);
+
+// Newton-DB stage-1 prologue: c = 1/(2 lambda); Y0 = c (F + eps I) (padding:
+// identity); D0 = (I - Y0)/2; Zhat1 = (I + D0)/zs; xscale = c^(1/4) zs.
+// D0 and Zhat1 are also written transposed (D0t, Z1t).
+void launch_ndb_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, float zs,
+                     __half* Y0, __half* D0, __half* D0t, __half* Z1, __half* Z1t, float* xscale,
+                     cudaStream_t st);
+
+// Newton-DB stage-2 prologue from the split Y of stage 1:
+// D0 = (I - Y)/2; Zhat1 = (I + D0)/zs; both also written transposed.
+void launch_ndb_stage2_init(const __half* Y, int nf, int B, float zs, __half* D0, __half* D0t, __half* Z1,
+                            __half* Z1t, cudaStream_t st);
+
+// out = xscale_f * Zhat (split in; fp32 and/or split out); used when a stage
+// has a single iteration.
+void launch_scale_split(const __half* Z, int nf, int B, const float* xscale, float* out_f32, __half* out_split,
+                        cudaStream_t st);
+
+// Chebyshev prologue with the spectral scaling c = 1/(2 lambda):
+// T = 2c (F + eps I) - I (padding: 0); b_{d-1} = c_{d-1} I + 2 c_d T;
+// xscale = c^(1/4).
+void launch_cheb_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda,
+                      float c_dm1, float c_d, __half* T, __half* bdm1, float* xscale, cudaStream_t st);
+
+// Gather gradient blocks into padded split matrices: Gs[2k] = G_k, Gs[2k+1] = G_k^T.
+void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int B, __half* Gs, cudaStream_t st);
+
+// factors[f] = init_scale * I.
+void launch_init_factors(float* F, int nf, int B, float init_scale, cudaStream_t st);
+
+// Adam moments and per-block sum of squares of the Adam direction P.
+void launch_adam(const ParamDev* params, const long long* item_prefix, int n_params, long long n_items, int B,
+                 float beta1, float beta2, float adam_eps, float bc1, float bc2, float* pnorm, cudaStream_t st);
+
+// param -= lr * sqrt(pnorm_k / unorm_k) * U (0 where unorm_k == 0).
+void launch_update(const ParamDev* params, const long long* item_prefix, int n_params, long long n_items, int B,
+                   float lr, const float* U, const float* pnorm, const float* unorm, cudaStream_t st);
+
+}  // namespace dash

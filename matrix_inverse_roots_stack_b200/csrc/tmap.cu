@@ -1,0 +1,45 @@
+#include "tmap.cuh"
+
+#include <mutex>
+
+namespace dash {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return cudaErrorInvalidValue;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || B % 128 != 0 || nmat < 1)
+    return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(B), static_cast<cuuint64_t>(B),
+                        static_cast<cuuint64_t>(2) * static_cast<cuuint64_t>(nmat)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(B) * 2u,
+                           static_cast<cuuint64_t>(B) * static_cast<cuuint64_t>(B) * 2u};
+  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t estride[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace dash

@@ -1,0 +1,17 @@
+// Host-side TMA tensor-map encoding.  The driver entry point is fetched
+// through the runtime (cudaGetDriverEntryPoint), so the library does not
+// link libcuda directly and can be loaded on a machine without a driver.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace dash {
+
+// Encode a 3-D tiled map over a split stack: dims {B (columns, innermost),
+// B (rows), 2 * nmat (matrix * 2 + plane)} of fp16, box {64, 128, 1},
+// 128-byte swizzle.  Returns cudaSuccess or cudaErrorInvalidValue.
+cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat);
+
+}  // namespace dash

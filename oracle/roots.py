@@ -88,11 +88,11 @@ def ndb_scalar(x, iters):
 
 
 def ndb_scale(lam_est):
-    """Spectral scaling c = 1/(2 lambda_est).
+    """Spectral scaling c = 1/(2 lambda_est), used by both solvers.
 
     DASH explainer, "Building blocks" (spectral scaling) and "Step-by-step"
-    (scale each block): divide the block by about 2*lambda_est.  Read
-    literally as the factor 2.
+    (scale each block, before the solver is chosen): divide the block by
+    about 2*lambda_est.  Read literally as the factor 2.
     """
     return 1.0 / (2.0 * float(lam_est))
 
@@ -180,15 +180,18 @@ def clenshaw_scalar(c, t):
 def cheb_phi(w, lam_est, degree, delta):
     """Scalar map of the Chebyshev inverse fourth root.
 
-    The spectrum is mapped into [delta, 1 + delta] by x = w/lambda_est + delta
-    (DASH explainer, "Step-by-step", solver (d): map the spectrum into
-    [eps, 1+eps]); the polynomial p ~ x^(-1/4) is evaluated at the Chebyshev
-    variable t = 2(x - delta) - 1 = 2 w/lambda_est - 1; the result is
-    lambda_est^(-1/4) p, which approximates (w + delta*lambda_est)^(-1/4).
+    DASH explainer, "Step-by-step": each block is first scaled by
+    c = 1/(2 lambda_est) (step "Scale each block using multi-Power-Iteration",
+    which precedes the choice of solver), then solver (d) maps the spectrum
+    into [delta, 1 + delta]: x = c w + delta.  The polynomial p ~ x^(-1/4) is
+    evaluated at the Chebyshev variable t = 2(x - delta) - 1 = 2 c w - 1, and
+    the scaling is undone: the result c^(1/4) p approximates
+    (w + delta / c)^(-1/4).
     """
-    c = cheb_inv4root_coeffs(degree, delta)
-    t = 2.0 * np.asarray(w, dtype=np.float64) / float(lam_est) - 1.0
-    return float(lam_est) ** -0.25 * clenshaw_scalar(c, t)
+    c = ndb_scale(lam_est)
+    cf = cheb_inv4root_coeffs(degree, delta)
+    t = 2.0 * c * np.asarray(w, dtype=np.float64) - 1.0
+    return c ** 0.25 * clenshaw_scalar(cf, t)
 
 
 def cheb_inv4root_spectral(A, lam_est, degree, delta):
@@ -201,17 +204,18 @@ def cheb_inv4root_spectral(A, lam_est, degree, delta):
 def cheb_inv4root_matmul(A, lam_est, degree, delta):
     """Level 3: the matrix Clenshaw recurrence with float64 products.
 
-    T = 2 A/lambda_est - I; b_k = c_k I + 2 T b_{k+1} - b_{k+2} for
-    k = d..1; p = c0/2 I + T b1 - b2; X = lambda_est^(-1/4) p.
+    c = 1/(2 lambda_est); T = 2 c A - I; b_k = c_k I + 2 T b_{k+1} - b_{k+2}
+    for k = d..1; p = c0/2 I + T b1 - b2; X = c^(1/4) p.
     """
     A = np.asarray(A, dtype=np.float64)
     n = A.shape[0]
     I = np.eye(n)
+    s = ndb_scale(lam_est)
     c = cheb_inv4root_coeffs(degree, delta)
-    T = 2.0 * A / float(lam_est) - I
+    T = 2.0 * s * A - I
     b1 = np.zeros((n, n))
     b2 = np.zeros((n, n))
     for k in range(degree, 0, -1):
         b1, b2 = c[k] * I + 2.0 * T @ b1 - b2, b1
     P = 0.5 * c[0] * I + T @ b1 - b2
-    return float(lam_est) ** -0.25 * P
+    return s ** 0.25 * P

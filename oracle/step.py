@@ -91,7 +91,8 @@ def inverse_fourth_root(Abar, V0, hp, lam_est=None):
             X = roots.ndb_inv4root_matmul(Abar, lam_est, hp.ndb_iters1, hp.ndb_iters2)
     elif hp.solver == "cheb":
         if hp.root_level == 1:
-            X = roots.inv_root_eigh(Abar + hp.cheb_delta * lam_est * np.eye(b), 4)
+            shift = hp.cheb_delta / roots.ndb_scale(lam_est)
+            X = roots.inv_root_eigh(Abar + shift * np.eye(b), 4)
         elif hp.root_level == 2:
             X = roots.cheb_inv4root_spectral(Abar, lam_est, hp.cheb_degree, hp.cheb_delta)
         else:

@@ -1,0 +1,139 @@
+"""GPU parity of the standalone inverse-root calls against the float64 oracle.
+
+Tolerances (relative Frobenius error per matrix): 1e-3 on inverse roots of
+matrices with condition number <= 1e6, against the truncated method evaluated
+exactly at the same power-iteration estimate (oracle level 2), and against
+the exact root (level 1) where level 2 has itself converged.
+"""
+
+import numpy as np
+import pytest
+
+from matrix_inverse_roots_stack_b200 import workloads
+from oracle import roots
+from tests.gpu_util import rel, cuda_or_skip
+
+pytestmark = pytest.mark.gpu
+
+ROOT_TOL = 1e-3
+LAMBDA_TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def torch():
+    return cuda_or_skip()
+
+
+def gpu_roots(torch, A, solver, eps=0.0, seed=0, pi_iters=10, **kw):
+    from matrix_inverse_roots_stack_b200 import binding as bd
+    B = A.shape[1]
+    v0 = workloads.pi_start_vectors(B, 32, seed=seed)
+    At = torch.from_numpy(np.ascontiguousarray(A, dtype=np.float32)).cuda()
+    vt = torch.from_numpy(v0).cuda()
+    if solver == "ndb":
+        X, lam, ws = bd.inv_root_newton_db(At, vt, eps=eps, pi_iters=pi_iters, **kw)
+    else:
+        X, lam, ws = bd.inv_root_chebyshev(At, vt, eps=eps, pi_iters=pi_iters, **kw)
+    rc, flags = bd.read_status(ws)
+    return X.cpu().numpy().astype(np.float64), lam.cpu().numpy().astype(np.float64), rc, v0
+
+
+def check_lambda(A, eps, lam, v0, pi_iters=10):
+    A64 = A.astype(np.float64)
+    for i in range(A.shape[0]):
+        Ab = A64[i] + eps * np.eye(A.shape[1])
+        lo, _ = roots.power_iteration(Ab, v0.astype(np.float64), pi_iters)
+        assert abs(lam[i] - lo) <= LAMBDA_TOL * lo, (i, lam[i], lo)
+        assert lam[i] <= np.linalg.eigvalsh(Ab)[-1] * (1 + 1e-5)
+
+
+def ndb_level2(A, eps, lam, t1, t2):
+    return [roots.ndb_inv4root_spectral(A[i].astype(np.float64) + eps * np.eye(A.shape[1]), lam[i], t1, t2)
+            for i in range(A.shape[0])]
+
+
+def cheb_level2(A, eps, lam, d, delta):
+    return [roots.cheb_inv4root_spectral(A[i].astype(np.float64) + eps * np.eye(A.shape[1]), lam[i], d, delta)
+            for i in range(A.shape[0])]
+
+
+def test_identity_closed_form(torch):
+    alpha = 2.5
+    A = np.stack([alpha * np.eye(128), 0.25 * np.eye(128)]).astype(np.float32)
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=14, iters2=14)
+    assert rc == 0
+    assert abs(lam[0] - alpha) < 1e-5 * alpha and abs(lam[1] - 0.25) < 1e-5 * 0.25
+    assert rel(X[0], alpha ** -0.25 * np.eye(128)) < 1e-5
+    assert rel(X[1], 0.25 ** -0.25 * np.eye(128)) < 1e-5
+
+
+def test_ndb_decaying_spectrum_converged(torch):
+    # the standalone-root workload's construction (kappa ~ 963), reduced count
+    A, U, lamv = workloads.spd_stack_decaying(n=6, b=256, seed=1)
+    X, lam, rc, v0 = gpu_roots(torch, A, "ndb", iters1=14, iters2=14)
+    assert rc == 0
+    check_lambda(A, 0.0, lam, v0)
+    ref2 = ndb_level2(A, 0.0, lam, 14, 14)
+    for i in range(6):
+        assert rel(X[i], ref2[i]) < ROOT_TOL
+        # level 2 converged here, so the exact root is within tolerance too
+        assert rel(X[i], roots.inv_root_eigh(A[i].astype(np.float64))) < ROOT_TOL
+
+
+@pytest.mark.parametrize("t1,t2", [(1, 1), (1, 3), (3, 1), (2, 2), (8, 8)])
+def test_ndb_iteration_counts(torch, t1, t2):
+    A = workloads.spd_stack_geometric(3, 256, 1e3, seed=2)
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=t1, iters2=t2, eps=1e-5)
+    assert rc == 0
+    for i, r in enumerate(ndb_level2(A, 1e-5, lam, t1, t2)):
+        assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
+
+
+def test_ndb_kappa_1e6(torch):
+    A = workloads.spd_stack_geometric(3, 128, 1e6, seed=3)
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=24, iters2=24)
+    assert rc == 0
+    for i, r in enumerate(ndb_level2(A, 0.0, lam, 24, 24)):
+        assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
+
+
+def test_ndb_many_tiles(torch):
+    # B = 512: 4 x 4 tiles (10 computed with the symmetric half), two matrices
+    A = workloads.spd_stack_geometric(2, 512, 1e4, seed=4, lam_max=37.0)
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=16, iters2=16, eps=1e-6)
+    assert rc == 0
+    for i, r in enumerate(ndb_level2(A, 1e-6, lam, 16, 16)):
+        assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
+
+
+@pytest.mark.parametrize("d,delta", [(2, 1e-3), (3, 1e-3), (16, 1e-3), (16, 1e-6), (40, 1e-3)])
+def test_chebyshev(torch, d, delta):
+    A = workloads.spd_stack_geometric(4, 256, 1e3, seed=5)
+    X, lam, rc, v0 = gpu_roots(torch, A, "cheb", degree=d, delta=delta, eps=1e-6)
+    assert rc == 0
+    check_lambda(A, 1e-6, lam, v0)
+    for i, r in enumerate(cheb_level2(A, 1e-6, lam, d, delta)):
+        assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
+
+
+def test_nonfinite_input_sets_status(torch):
+    from matrix_inverse_roots_stack_b200 import binding as bd
+    A = workloads.spd_stack_geometric(2, 128, 10.0, seed=6)
+    A[1, 3, 3] = np.nan
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=2, iters2=2)
+    assert rc == bd.SHAMPOO_ENONFINITE
+
+
+def test_standalone_workload_full_size(torch):
+    # 256 SPD blocks of 256 (decaying spectrum, kappa ~ 963): Newton-DB 14+14
+    # and Chebyshev degree 16, every matrix compared
+    A, _, _ = workloads.spd_stack_decaying(n=256, b=256, seed=0)
+    X, lam, rc, v0 = gpu_roots(torch, A, "ndb", iters1=14, iters2=14)
+    assert rc == 0
+    check_lambda(A[:8], 0.0, lam[:8], v0)
+    errs = [rel(X[i], r) for i, r in enumerate(ndb_level2(A, 0.0, lam, 14, 14))]
+    assert max(errs) < ROOT_TOL, max(errs)
+    X, lam, rc, _ = gpu_roots(torch, A, "cheb", degree=16, delta=1e-3)
+    assert rc == 0
+    errs = [rel(X[i], r) for i, r in enumerate(cheb_level2(A, 0.0, lam, 16, 1e-3))]
+    assert max(errs) < ROOT_TOL, max(errs)

@@ -205,7 +205,8 @@ def test_cheb_matrix_diagonal_matches_chebval():
     c = roots.cheb_inv4root_coeffs(d, delta)
     cc = c.copy()
     cc[0] *= 0.5
-    expect = npcheb.chebval(2.0 * w / lam - 1.0, cc) * lam ** -0.25
+    # spectral scaling 1/(2 lam): t = w/lam - 1, undone by (2 lam)^(-1/4)
+    expect = npcheb.chebval(w / lam - 1.0, cc) * (2.0 * lam) ** -0.25
     assert rel(np.diag(X), expect) < 1e-13
 
 
@@ -218,12 +219,21 @@ def test_cheb_level2_matches_level3():
 
 
 def test_cheb_high_degree_approaches_shifted_target():
-    # p approximates x^(-1/4) on [delta, 1+delta]; the matrix result is
-    # lam^(-1/4) p(A/lam + delta) ~ (A + delta*lam I)^(-1/4)
+    # p approximates x^(-1/4) on [delta, 1+delta]; with c = 1/(2 lam) the
+    # matrix result c^(1/4) p(c A + delta I) ~ (A + 2 delta lam I)^(-1/4)
     A, _, w = random_spd(24, 50.0, seed=10)
     lam, delta = w.max(), 0.05
     X = roots.cheb_inv4root_spectral(A, lam, 40, delta)
-    assert rel(X, roots.inv_root_eigh(A + delta * lam * np.eye(24))) < 1e-9
+    assert rel(X, roots.inv_root_eigh(A + 2.0 * delta * lam * np.eye(24))) < 1e-9
+
+
+def test_cheb_spectrum_stays_inside_interval():
+    # with the 1/(2 lam) scaling an estimate up to 2x below lam_max still maps
+    # the spectrum into [delta, 1 + delta], i.e. t in [-1, 1]
+    w = np.linspace(1e-3, 1.0, 50)
+    for lam in (1.0, 0.9, 0.5):
+        t = 2.0 * roots.ndb_scale(lam) * w - 1.0
+        assert t.min() >= -1.0 and t.max() <= 1.0
 
 
 # ---------------------------------------------------------------- power iteration

@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of one batched block-Shampoo (DASH-style) optimizer step on B200.
+
+Default workload: a ~1B Llama-shaped parameter set (24 layers, d=2048, SwiGLU
+MLP 2048x5632 x3, embedding and head 32000x2048), fp32 gradients N(0, 1e-2)
+with a per-row LogNormal(0, 1) scale, block size B=1024, every step
+preconditioned: factor EMA, 10 power-iteration products from 32 starts,
+Newton-DB 14 + 14 iterations (or Chebyshev), preconditioning, Adam graft and
+update.  Inputs are synthetic (seeded) and resident in HBM; the working set
+(~100 GB) is far larger than L2, so no L2 flush is needed between steps.
+
+One JSON line on rank 0: the step time (ms, lower is better), the roofline of
+the dominant kernel (the tensor-core GEMM, per-launch CUDA-event durations
+measured inside the timed region), the root-stage TFLOP/s as a fraction of the
+dense TF32 peak, an end-to-end figure through the C ABI with host buffers, the
+SM clocks sampled during the timed region, and the float64 oracle timed on the
+host cores on a bounded sample of the same workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload llama1b|gpt2|spiked512|roots256|mixed]
+
+For N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the workload (weak scaling; the blocks of different ranks are independent
+problems and no collective is on the data path); the step time is the max
+over ranks.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="llama1b",
+                   choices=["llama1b", "gpt2", "spiked512", "roots256", "mixed"])
+    p.add_argument("--block", type=int, default=None, help="override the block size")
+    p.add_argument("--solver", default="ndb", choices=["ndb", "cheb"])
+    p.add_argument("--iters", type=int, default=None, help="Newton-DB iterations per stage")
+    p.add_argument("--degree", type=int, default=16)
+    p.add_argument("--n", type=int, default=256, help="matrices in the standalone-roots workload")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------
+# workloads
+# --------------------------------------------------------------------------
+
+def workload_spec(args):
+    from matrix_inverse_roots_stack_b200 import workloads as wl
+    if args.workload == "llama1b":
+        spec = dict(shapes=wl.llama_1b_shapes(), B=1024, grad="lognormal", iters=14,
+                    desc="llama-1b-shaped param set (24 layers, d=2048, SwiGLU 2048x5632 x3, "
+                         "embed+head 32000x2048), fp32 grads N(0,1e-2) x row LogNormal(0,1)")
+    elif args.workload == "gpt2":
+        spec = dict(shapes=wl.gpt2_124m_shapes(), B=512, grad="gauss", iters=14,
+                    desc="gpt2-124m-shaped param set (12 layers, d=768, QKV 768x2304, attn-out, "
+                         "MLP 768x3072/3072x768, wte 50257x768, wpe 1024x768), fp32 grads N(0,1e-2)")
+    elif args.workload == "spiked512":
+        spec = dict(shapes=[(512, 512)], B=128, grad="spiked", iters=8,
+                    desc="single 512x512 fp32 weight, gradient N(0,1) + rank-8 spike (scale 10)")
+    elif args.workload == "mixed":
+        spec = dict(shapes=wl.mixed_shapes(), B=1024, grad="student", iters=14,
+                    desc="mixed shapes 1024x4096, 4096x1024, 2048x2048, Student-t(3) grads")
+    else:
+        spec = dict(shapes=None, B=256, grad=None, iters=14, n=args.n,
+                    desc=f"standalone inverse 4th roots: {args.n} SPD blocks, A = G G^T/1024 + 1e-6 I, "
+                         "singular values of G decaying as 1/k")
+    if args.block:
+        spec["B"] = args.block
+    if args.iters:
+        spec["iters"] = args.iters
+    return spec
+
+
+def make_grads(spec, device, seed=0):
+    import torch
+    from matrix_inverse_roots_stack_b200 import workloads as wl
+    if spec["grad"] == "lognormal":
+        return wl.torch_gaussian_gradients(spec["shapes"], device, std=0.1, seed=seed, row_lognormal_sigma=1.0)
+    if spec["grad"] == "gauss":
+        return wl.torch_gaussian_gradients(spec["shapes"], device, std=0.1, seed=seed)
+    if spec["grad"] == "student":
+        return wl.torch_student_t_gradients(spec["shapes"], device, nu=3.0, seed=seed)
+    if spec["grad"] == "spiked":
+        return [torch.from_numpy(wl.spiked_gradient(512, 512, rank=8, scale=10.0, seed=seed)).to(device)]
+    raise ValueError(spec["grad"])
+
+
+def block_sizes(shapes, B):
+    out = []
+    for (r, c) in shapes:
+        for r0 in range(0, r, B):
+            for c0 in range(0, c, B):
+                out.append((min(B, r - r0), min(B, c - c0)))
+    return out
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# CPU baseline / reference arm: the float64 oracle on a bounded sample
+# --------------------------------------------------------------------------
+
+def oracle_sample(spec, args, budget_s=15.0, seed=0):
+    """Time the oracle step on the first blocks of the workload until about
+    budget_s seconds of CPU work; returns (ms per full step extrapolated by
+    block count, description, threads)."""
+    import numpy as np
+    from oracle import step as ostep, roots
+    from matrix_inverse_roots_stack_b200 import workloads as wl
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    B = spec["B"]
+    iters = spec["iters"]
+    hp = ostep.HParams(block_size=B, ndb_iters1=iters, ndb_iters2=iters,
+                       solver="ndb" if args.solver == "ndb" else "cheb", cheb_degree=args.degree)
+    V0 = wl.pi_start_vectors(B, 32, seed=0).astype(np.float64)
+    if spec["shapes"] is None:  # standalone roots: time per matrix
+        nmat = spec.get("n", 256)
+        A, _, _ = wl.spd_stack_decaying(n=min(4, nmat), b=B, seed=seed)
+        t0 = time.perf_counter()
+        done = 0
+        for i in range(A.shape[0]):
+            lam, _ = roots.power_iteration(A[i].astype(np.float64), V0, 10)
+            roots.ndb_inv4root_spectral(A[i].astype(np.float64), lam, iters, iters)
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return (dt / done * nmat * 1e3, f"{done} of {nmat} matrices ({B}x{B}), extrapolated x{nmat / done:.1f}",
+                threads)
+    shapes = spec["shapes"]
+    total_blocks = len(block_sizes(shapes, B))
+    rng = np.random.default_rng(seed)
+    t0 = time.perf_counter()
+    done_blocks, used = 0, []
+    for (r, c) in shapes:
+        G = rng.standard_normal((r, c)) * 0.1
+        th = np.zeros((r, c))
+        state = ostep.init_state([(r, c)], hp)
+        ostep.shampoo_step([th], [G], state, hp, V0)
+        done_blocks += len(block_sizes([(r, c)], B))
+        used.append(f"{r}x{c}")
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    frac = total_blocks / done_blocks
+    return (dt * frac * 1e3, f"oracle step (level 2, eigh) on parameters {', '.join(used)} = {done_blocks} of "
+            f"{total_blocks} blocks, extrapolated x{frac:.1f} by block count", threads)
+
+
+def run_reference(args, spec, rank):
+    if rank != 0:
+        return
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        ms, sample, threads = oracle_sample(spec, args, budget_s=8.0)
+        if i >= args.warmup:
+            per_step.append(ms)
+    ms = statistics.median(per_step)
+    line = {"impl": "reference", "metric": "Shampoo optimizer step ms", "value": round(ms, 3), "unit": "ms",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": spec["desc"], "block_size": spec["B"],
+                                            "solver": args.solver, "iters": spec["iters"]},
+            "cpu_baseline": {"value": round(ms, 3), "unit": "ms", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def main():
+    args = parse_args()
+    spec = workload_spec(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, spec, rank)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    from matrix_inverse_roots_stack_b200 import binding as bd, build, workloads as wl
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    B = spec["B"]
+    iters = spec["iters"]
+    solver = bd.SOLVER_NEWTON_DB if args.solver == "ndb" else bd.SOLVER_CHEBYSHEV
+    stream = torch.cuda.current_stream()
+
+    if spec["shapes"] is None:
+        # standalone roots workload
+        nmat = spec["n"]
+        A, _, _ = wl.spd_stack_decaying(n=nmat, b=B, seed=0)
+        At = torch.from_numpy(A).to(dev)
+        X = torch.empty_like(At)
+        lam = torch.empty(nmat, dtype=torch.float32, device=dev)
+        v0 = torch.from_numpy(wl.pi_start_vectors(B, 32, seed=0)).to(dev)
+        need = bd.inv_root_workspace_bytes(nmat, B, solver)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+        def step_fn():
+            if solver == bd.SOLVER_NEWTON_DB:
+                bd.inv_root_newton_db(At, v0, iters, iters, 0.0, 10, X, lam, ws)
+            else:
+                bd.inv_root_chebyshev(At, v0, args.degree, 1e-3, 0.0, 10, X, lam, ws)
+        n_factors, factor_sizes = nmat, [B] * nmat
+        ctx_info = {"n_matrices": nmat}
+        e2e_fn = None
+    else:
+        grads = make_grads(spec, dev, seed=0)
+        params = [torch.randn(g.shape, device=dev) * 0.02 for g in grads]
+        hp = bd.make_hparams(block_size=B, solver=solver, ndb_iters1=iters, ndb_iters2=iters,
+                             cheb_degree=args.degree)
+        opt = bd.Shampoo(params, grads, hp=hp,
+                         v0=torch.from_numpy(wl.pi_start_vectors(B, 32, seed=0)).to(dev))
+        bsz = block_sizes(spec["shapes"], B)
+        factor_sizes = [s for pair in bsz for s in pair]
+        n_factors = opt.n_factors
+        ctx_info = {"n_params": len(params), "n_blocks": opt.n_blocks, "n_factors": opt.n_factors,
+                    "workspace_gb": round(opt.ws.numel() / 1e9, 2)}
+
+        def step_fn():
+            opt.step()
+
+        def e2e_fn(host_g, host_p):
+            # the same step through the C ABI with host buffers: upload the
+            # step's gradients from pinned memory, step, read the parameters back
+            off = 0
+            for g in grads:
+                n = g.numel()
+                g.view(-1).copy_(host_g[off:off + n], non_blocking=True)
+                off += n
+            opt.step()
+            off = 0
+            for p in params:
+                n = p.numel()
+                host_p[off:off + n].copy_(p.view(-1), non_blocking=True)
+                off += n
+
+    # ---------------- warm-up
+    for _ in range(args.warmup):
+        step_fn()
+    torch.cuda.synchronize()
+    if spec["shapes"] is not None:
+        rc, flags = opt.status()
+        if rc != 0:
+            print(f"[bench] warning: status {bd.strerror(rc)} (flags {flags})", file=sys.stderr)
+
+    # ---------------- timed region
+    bd.profile_reset()
+    bd.profile_enable(True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step_fn()
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    bd.profile_enable(False)
+    prof = bd.profile_read()
+    ms = t_start.elapsed_time(t_stop) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---------------- end to end through host buffers
+    e2e = None
+    if e2e_fn is not None and not args.no_e2e:
+        n_g = sum(g.numel() for g in grads)
+        n_p = sum(p.numel() for p in params)
+        try:
+            host_g = torch.empty(n_g, dtype=torch.float32, pin_memory=True)
+            host_p = torch.empty(n_p, dtype=torch.float32, pin_memory=True)
+            off = 0
+            for g in grads:
+                host_g[off:off + g.numel()].copy_(g.view(-1).cpu())
+                off += g.numel()
+            e2e_fn(host_g, host_p)
+            torch.cuda.synchronize()
+            barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                e2e_fn(host_g, host_p)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            e_ms = e0.elapsed_time(e1) / args.steps
+            if world > 1:
+                t = torch.tensor([e_ms], device=dev)
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+                e_ms = float(t.item())
+            e2e = {"value": round(e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 4 * n_g,
+                   "d2h_bytes_per_step": 4 * n_p}
+            del host_g, host_p
+        except RuntimeError as exc:
+            e2e = {"value": None, "unit": "ms", "error": str(exc)[:200]}
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # ---------------- roofline of the dominant kernel (the split-fp16 GEMM)
+    peaks, peak_kind = load_peaks()
+    g_ms, g_n, g_flops = prof["gemm"]
+    tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    avg_ms = g_ms / max(g_n, 1)
+    # 3 fp16 MMA products (hi*hi, hi*lo, lo*hi) per useful product
+    achieved = 3.0 * (g_flops / max(g_n, 1)) / (avg_ms * 1e-3) / 1e12 if g_n else None
+    roofline = {"kernel": "gemm_split_kernel", "bound": "tensor",
+                "achieved": round(achieved, 1) if achieved else None, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4) if achieved else None,
+                "traffic": None, "peak_kind": f"{peak_kind} bf16/fp16 dense, sustained",
+                "launches": g_n, "avg_launch_ms": round(avg_ms, 4),
+                "share_of_step": round(g_ms / (ms * args.steps), 4)}
+
+    # ---------------- root-stage TFLOP/s vs dense TF32 peak
+    s_ms = prof["solver"][0] + prof["power_iteration"][0]
+    if args.solver == "ndb":
+        gemms = 2 * (3 * iters - 3)            # both stages, first-iteration and last-iteration savings
+    else:
+        gemms = args.degree - 1
+    padded = 2.0 * B ** 3 * gemms * n_factors
+    unpadded = sum(2.0 * b ** 3 * gemms for b in factor_sizes)
+    tf32_peak = tensor_peak / 2.0
+    root_s = s_ms * 1e-3 / args.steps
+    inverse_root = {"ms_per_step": round(root_s * 1e3, 3),
+                    "tflops": round(padded / root_s / 1e12, 1),
+                    "tflops_unpadded": round(unpadded / root_s / 1e12, 1),
+                    "tf32_peak_tflops": tf32_peak,
+                    "frac_of_tf32_peak": round(padded / root_s / 1e12 / tf32_peak, 4),
+                    "frac_of_tf32_peak_unpadded": round(unpadded / root_s / 1e12 / tf32_peak, 4),
+                    "peak_kind": f"{peak_kind}: bf16 sustained x 0.5 (nominal TF32/BF16 ratio)"}
+    stages = {k: round(v[0] / args.steps, 3) for k, v in prof.items() if isinstance(v, tuple) and k != "gemm"}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        c_ms, sample, threads = oracle_sample(spec, args, budget_s=15.0)
+        cpu = {"value": round(c_ms, 1), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample}
+
+    line = {"metric": "Shampoo optimizer step ms", "value": round(ms, 3), "unit": "ms", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (3 x fp16-split tensor products, fp32 accumulate)",
+            "data": "synthetic",
+            "config": dict({"workload": spec["desc"], "block_size": B, "solver": args.solver,
+                            "iters_per_stage": iters if args.solver == "ndb" else None,
+                            "cheb_degree": args.degree if args.solver == "cheb" else None,
+                            "power_iteration": "10 products x 32 starts",
+                            "l2": "working set far larger than the 126 MB L2 (no flush needed)",
+                            "parallelism": f"replicas x{world}"}, **ctx_info),
+            "roofline": roofline, "inverse_root": inverse_root, "stage_ms": stages,
+            "gpu_launches": prof["launches"], "clocks": clock_info, "e2e": e2e, "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -167,6 +167,35 @@ SHAMPOO_API int shampoo_inv_root_chebyshev(const float* A, float* X, int n, int 
                                const float* v0, int pi_iters, float* lambda_out, void* ws, size_t ws_bytes,
                                void* stream);
 
+/* Variant of shampoo_inv_root_newton_db that allocates nothing and needs no
+ * workspace from the caller.  The paper has no counterpart: this exists for
+ * callers that cannot call cudaMalloc -- e.g. a plug-in running inside a host
+ * framework that owns every device allocation, or a latency-critical path
+ * where an allocation (which may synchronise the device) is not allowed.
+ *
+ * The scratch is a fixed array of SHAMPOO_STATIC_SCRATCH_BYTES in the
+ * library's device global memory; every GPU that loads the library holds it
+ * until the process exits.  Problems whose workspace
+ * (shampoo_inv_root_workspace_bytes(n, B, SHAMPOO_SOLVER_NEWTON_DB)) exceeds it
+ * are rejected with SHAMPOO_EWORKSPACE (it holds up to 112 matrices of 128,
+ * 30 of 256, 7 of 512, 1 of 1024).  The caller still passes A, X, v0 and lambda_out (device
+ * pointers, as for shampoo_inv_root_newton_db); the computation and the
+ * results are the same.
+ *
+ * The first call on a device looks up the scratch's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents (each call clears what must start at zero), so calls whose GPU work
+ * overlaps -- on different streams, or from different threads -- race on it:
+ * serialise them.  The status word lives in the scratch too and is cleared at
+ * each call; it is not readable through this entry point.
+ * Errors: as shampoo_inv_root_newton_db, plus SHAMPOO_EWORKSPACE when the
+ * problem does not fit the scratch. */
+#define SHAMPOO_STATIC_SCRATCH_BYTES (64u << 20)
+SHAMPOO_API int shampoo_inv_root_newton_db_static(const float* A, float* X, int n, int B, int iters1, int iters2,
+                                                  float eps, const float* v0, int pi_iters, float* lambda_out,
+                                                  void* stream);
+
 /* Workspace bytes for a standalone root call on n matrices of size B. */
 SHAMPOO_API size_t shampoo_inv_root_workspace_bytes(int n, int B, int solver);
 

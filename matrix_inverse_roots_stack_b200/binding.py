@@ -68,6 +68,7 @@ _PROTOS = {
     "shampoo_read_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_uint)]),
     "shampoo_strerror": (ctypes.c_char_p, [_I]),
     "shampoo_destroy": (None, [_VP]),
+    "shampoo_inv_root_newton_db_static": (_I, [_VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _VP, _VP]),
     "shampoo_profile_enable": (_I, [_I]),
     "shampoo_profile_reset": (_I, []),
     "shampoo_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), _I]),
@@ -157,6 +158,23 @@ def inv_root_chebyshev(A, v0, degree=16, delta=1e-3, eps=0.0, pi_iters=10, X=Non
                                            _ptr(lam), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "shampoo_inv_root_chebyshev")
     return X, lam, ws
+
+
+STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def inv_root_newton_db_static(A, v0, iters1=14, iters2=14, eps=0.0, pi_iters=10, X=None, lam=None, stream=None):
+    """:func:`inv_root_newton_db` through the entry point that uses the
+    library's fixed scratch instead of a workspace (nothing is allocated by
+    the library; X and lambda are allocated here only if not given)."""
+    import torch
+    n, B = A.shape[0], A.shape[1]
+    X = torch.empty_like(A) if X is None else X
+    lam = torch.empty(n, dtype=torch.float32, device=A.device) if lam is None else lam
+    rc = load().shampoo_inv_root_newton_db_static(_ptr(A), _ptr(X), n, B, iters1, iters2, eps, _ptr(v0), pi_iters,
+                                                  _ptr(lam), _stream(stream))
+    _check(rc, "shampoo_inv_root_newton_db_static")
+    return X, lam
 
 
 def read_status(ws, stream=None):

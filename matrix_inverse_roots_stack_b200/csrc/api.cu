@@ -687,3 +687,16 @@ const char* shampoo_strerror(int code) {
 void shampoo_destroy(shampoo_ctx* ctx) { delete ctx; }
 
 }  // extern "C"
+
+namespace dash {
+
+// Standalone root computation on a caller-provided scratch region (used by
+// the static-scratch entry point in noalloc.cu).
+int inv_root_with_scratch(const float* A, float* X, int n, int B, float eps, const float* v0, int pi_iters, void* ws,
+                          size_t ws_bytes, int solver, int it1, int it2, int degree, float delta, float* lambda_out,
+                          void* stream) {
+  return inv_root_common(A, X, n, B, eps, v0, pi_iters, ws, ws_bytes, solver, it1, it2, degree, delta, lambda_out,
+                         stream);
+}
+
+}  // namespace dash

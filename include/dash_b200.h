@@ -177,8 +177,8 @@ SHAMPOO_API int shampoo_inv_root_chebyshev(const float* A, float* X, int n, int 
  * library's device global memory; every GPU that loads the library holds it
  * until the process exits.  Problems whose workspace
  * (shampoo_inv_root_workspace_bytes(n, B, SHAMPOO_SOLVER_NEWTON_DB)) exceeds it
- * are rejected with SHAMPOO_EWORKSPACE (it holds up to 112 matrices of 128,
- * 30 of 256, 7 of 512, 1 of 1024).  The caller still passes A, X, v0 and lambda_out (device
+ * are rejected with SHAMPOO_EWORKSPACE (it holds up to 168 matrices of 128,
+ * 47 of 256, 12 of 512, 3 of 1024).  The caller still passes A, X, v0 and lambda_out (device
  * pointers, as for shampoo_inv_root_newton_db); the computation and the
  * results are the same.
  *
@@ -200,7 +200,8 @@ SHAMPOO_API int shampoo_inv_root_newton_db_static(const float* A, float* X, int 
 SHAMPOO_API size_t shampoo_inv_root_workspace_bytes(int n, int B, int solver);
 
 /* Synchronise `stream`, read the status word of `ws` into *flags (host, may
- * be NULL) and return SHAMPOO_OK, SHAMPOO_ENONFINITE or SHAMPOO_ETIMEOUT. */
+ * be NULL) and return SHAMPOO_OK, SHAMPOO_ETIMEOUT (checked first: a wait
+ * that gave up leaves later results undefined) or SHAMPOO_ENONFINITE. */
 SHAMPOO_API int shampoo_read_status(const void* ws, void* stream, unsigned* flags);
 
 /* Static description of a status code. */
@@ -222,6 +223,14 @@ SHAMPOO_API int shampoo_profile_reset(void);
  * products, 5 Adam graft + update; out[18] = kernel launches since the last
  * reset; out[19] = records dropped. */
 SHAMPOO_API int shampoo_profile_read(double* out, int n);
+
+/* Test hook for the failure path (not part of the method): arms a one-shot
+ * fault so that the next tensor-core GEMM launch withholds its operand
+ * loads.  Its bounded waits then expire (about 2 s), the kernel sets
+ * SHAMPOO_STATUS_TIMEOUT in the workspace status word, releases its tensor
+ * memory and returns; the context stays usable.  The results of that call
+ * are undefined. */
+SHAMPOO_API int shampoo_debug_inject_timeout(void);
 
 /* Free a ctx (host memory only).  NULL is ignored. */
 SHAMPOO_API void shampoo_destroy(shampoo_ctx* ctx);

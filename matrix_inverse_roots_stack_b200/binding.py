@@ -69,6 +69,7 @@ _PROTOS = {
     "shampoo_strerror": (ctypes.c_char_p, [_I]),
     "shampoo_destroy": (None, [_VP]),
     "shampoo_inv_root_newton_db_static": (_I, [_VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _VP, _VP]),
+    "shampoo_debug_inject_timeout": (_I, []),
     "shampoo_profile_enable": (_I, [_I]),
     "shampoo_profile_reset": (_I, []),
     "shampoo_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), _I]),

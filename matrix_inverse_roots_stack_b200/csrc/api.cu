@@ -37,10 +37,11 @@ struct Bump {
   }
 };
 
-// Factors per solver chunk: the Newton-DB scratch is 8 split matrices per
-// factor, bounded by kSolverBudget.
+// Factors per solver chunk: the Newton-DB scratch is 5 split matrices per
+// factor (Chebyshev needs 4), bounded by kSolverBudget.
+constexpr int kSolverMats = 5;
 int solver_chunk(int nf, int B) {
-  const size_t per = 8u * split_bytes(1, B);
+  const size_t per = kSolverMats * split_bytes(1, B);
   size_t m = kSolverBudget / per;
   if (m < 1) m = 1;
   return static_cast<int>(m < static_cast<size_t>(nf) ? m : nf);
@@ -60,7 +61,7 @@ void plan_roots(Bump& b, RootLayout& L, int nf, int B, int pi_iters, int extra_m
   L.w0 = b.take(sizeof(float) * static_cast<size_t>(nf) * B * dash::kPiStarts);
   L.w1 = b.take(sizeof(float) * static_cast<size_t>(nf) * B * dash::kPiStarts);
   L.chunk = solver_chunk(nf, B);
-  const int mats = 8 * L.chunk > extra_mats ? 8 * L.chunk : extra_mats;
+  const int mats = kSolverMats * L.chunk > extra_mats ? kSolverMats * L.chunk : extra_mats;
   L.solver = b.take(split_bytes(mats, B));
 }
 
@@ -116,46 +117,42 @@ GemmArgs gemm_args(int B, int sym, unsigned* status) {
 // left): in finite precision that is the stable form of the coupled
 // iteration, while symmetrising an iterate or moving Z's factor to the other
 // side makes a perturbation mode grow once the condition number exceeds ~10.
-// Every product is therefore a full (non-symmetric) product; since both
-// operands are read K-major, each iterate is kept together with its
-// transpose: P = Z Y uses (Z, Y^T), Y E uses (Y, E^T) and E Z is formed as
-// its transpose Z^T E^T from (Z^T, E).  E = I + D is applied in correction
-// form Y + Y D, Z + D Z.  Z is stored divided by kZScale.
+// Every product is therefore a full (non-symmetric) product of the iterates in
+// their natural layout (the GEMM reads the right factor MN-major).  E = I + D
+// is applied in correction form Y + Y D, Z + D Z.  Z is stored divided by
+// kZScale.  Scratch: Y x2, Z x2 (ping-pong), D: 5 split matrices per factor.
 int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, const float* lam, float* xscale,
                   int it1, int it2, float* X_f32, __half* X_split, __half* S, unsigned* status,
                   cudaStream_t st) {
   const size_t m = static_cast<size_t>(n) * 2 * B * B;  // halves per buffer of n matrices
   __half* Yb[2] = {S, S + m};
-  __half* Yt = S + 2 * m;
-  __half* Z = S + 3 * m;
-  __half* Zt[2] = {S + 4 * m, S + 5 * m};
-  __half* D = S + 6 * m;
-  __half* Dt = S + 7 * m;
-  dash::launch_ndb_init(F, n, B, eps, fsize, lam, kZScale, Yb[0], D, Dt, Z, Zt[0], xscale, st);
-  DASH_LAUNCHED();
+  __half* Zb[2] = {S + 2 * m, S + 3 * m};
+  __half* D = S + 4 * m;
   int yc = 0, zc = 0;
+  dash::launch_ndb_init(F, n, B, eps, fsize, lam, kZScale, Yb[0], D, Zb[0], xscale, st);
+  DASH_LAUNCHED();
 
-  // Y <- Y + Y D  (A = Y, Bm = D^T); also writes Y^T
+  // Y <- Y + Y D  (A = Y, B = D)
   auto y_op = [&](GemmArgs& g, dash::OpBuffers* ob, int slot) {
     dash::GemmOp& o = g.op[slot];
     o.nprob = n;
+    o.b_mn = 1;
     o.alpha = 1.0f;
     o.beta = 1.0f;
     o.cin_split = Yb[yc];
     o.out_split = Yb[yc ^ 1];
-    o.outt_split = Yt;
-    ob[slot] = {Yb[yc], n, Dt, n};
+    ob[slot] = {Yb[yc], n, D, n};
   };
-  // Z^T <- Z^T + Z^T D^T  (A = Z^T, Bm = D); writes Z^T and, transposed, Z
+  // Z <- Z + D Z  (A = D, B = Z)
   auto z_op = [&](GemmArgs& g, dash::OpBuffers* ob, int slot) {
     dash::GemmOp& o = g.op[slot];
     o.nprob = n;
+    o.b_mn = 1;
     o.alpha = 1.0f;
     o.beta = 1.0f;
-    o.cin_split = Zt[zc];
-    o.out_split = Zt[zc ^ 1];
-    o.outt_split = Z;
-    ob[slot] = {Zt[zc], n, D, n};
+    o.cin_split = Zb[zc];
+    o.out_split = Zb[zc ^ 1];
+    ob[slot] = {D, n, Zb[zc], n};
   };
   auto first_y = [&]() -> int {
     GemmArgs g = gemm_args(B, 0, status);
@@ -167,21 +164,21 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
   };
   auto iterate = [&](int T, bool final_stage) -> int {
     for (int it = 1; it < T; ++it) {
-      {  // D = (I - zs Zhat Y)/2 and D^T   (A = Zhat, Bm = Y^T)
+      {  // D = (I - zs Zhat Y)/2   (A = Zhat, B = Y)
         GemmArgs g = gemm_args(B, 0, status);
         dash::GemmOp& o = g.op[0];
         o.nprob = n;
+        o.b_mn = 1;
         o.alpha = -0.5f * kZScale;
         o.gamma = 0.5f;
         o.out_split = D;
-        o.outt_split = Dt;
-        dash::OpBuffers ob[2] = {{Z, n, Yt, n}, {Z, n, Yt, n}};
+        dash::OpBuffers ob[2] = {{Zb[zc], n, Yb[yc], n}, {Zb[zc], n, Yb[yc], n}};
         DASH_TRY(dash::launch_gemm_split(ob, g, st));
       }
       const bool last = (it == T - 1);
       GemmArgs g = gemm_args(B, 0, status);
       dash::OpBuffers ob[2];
-      if (!last) {
+      if (!last) {  // both updates in one launch
         y_op(g, ob, 0);
         z_op(g, ob, 1);
         g.nops = 2;
@@ -192,12 +189,11 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
         y_op(g, ob, 0);
         DASH_TRY(dash::launch_gemm_split(ob, g, st));
         yc ^= 1;
-      } else {  // X = c^(1/4) zs (Zhat + D Zhat), written in normal orientation
+      } else {  // X = c^(1/4) zs (Zhat + D Zhat)
         z_op(g, ob, 0);
         dash::GemmOp& o = g.op[0];
-        o.out_split = nullptr;
-        o.outt_split = X_split;
-        o.outt_f32 = X_f32;
+        o.out_split = X_split;
+        o.out_f32 = X_f32;
         o.scale = xscale;
         DASH_TRY(dash::launch_gemm_split(ob, g, st));
       }
@@ -210,10 +206,10 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
   rc = iterate(it1, false);
   if (rc) return rc;
   // stage 2 on Y: D0 = (I - Y)/2, Zhat1 = (I + D0)/zs, Y1 = Y + Y D0
-  dash::launch_ndb_stage2_init(Yb[yc], n, B, kZScale, D, Dt, Z, Zt[zc], st);
+  dash::launch_ndb_stage2_init(Yb[yc], n, B, kZScale, D, Zb[zc], st);
   DASH_LAUNCHED();
   if (it2 == 1) {
-    dash::launch_scale_split(Z, n, B, xscale, X_f32, X_split, st);
+    dash::launch_scale_split(Zb[zc], n, B, xscale, X_f32, X_split, st);
     DASH_LAUNCHED();
     return SHAMPOO_OK;
   }
@@ -574,23 +570,25 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   __half* Gs = split_at(ws, ctx->off_gs, 0, B);
   __half* T1 = split_at(ws, ctx->roots.solver, 0, B);  // the solver scratch is free now
   const int uslot = dash::prof_begin(dash::kProfPrecond, st);
-  {  // T1_k^T = (G_k X_R)^T   (A = G_k, Bm = X_R, symmetric)
+  {  // T1_k = G_k X_R   (A = G_k, B = X_R)
     GemmArgs g = gemm_args(B, 0, status);
     dash::GemmOp& o = g.op[0];
     o.nprob = nb;
     o.a.stride = 2;
     o.b.base = 1;
     o.b.stride = 2;
+    o.b_mn = 1;
     o.alpha = 1.0f;
-    o.outt_split = T1;
+    o.out_split = T1;
     dash::OpBuffers ob[2] = {{Gs, nf, roots, nf}, {Gs, nf, roots, nf}};
     DASH_TRY(dash::launch_gemm_split(ob, g, st));
   }
-  {  // U_k = X_L T1_k, scattered into parameter layout with ||U_k||^2
+  {  // U_k = X_L T1_k, scattered into parameter layout with ||U_k||^2   (A = X_L, B = T1_k)
     GemmArgs g = gemm_args(B, 0, status);
     dash::GemmOp& o = g.op[0];
     o.nprob = nb;
     o.a.stride = 2;
+    o.b_mn = 1;
     o.alpha = 1.0f;
     o.blocks = reinterpret_cast<const BlockDesc*>(ws + ctx->off_blocks);
     o.u_out = U;
@@ -666,8 +664,8 @@ int shampoo_read_status(const void* ws, void* stream, unsigned* flags) {
   unsigned w = 0;
   DASH_TRY(cudaMemcpy(&w, ws, sizeof(unsigned), cudaMemcpyDeviceToHost));
   if (flags) *flags = w;
+  if (w & dash::kStatusTimeout) return SHAMPOO_ETIMEOUT;  // the root cause when both are set
   if (w & dash::kStatusNonFinite) return SHAMPOO_ENONFINITE;
-  if (w & dash::kStatusTimeout) return SHAMPOO_ETIMEOUT;
   return SHAMPOO_OK;
 }
 
@@ -685,6 +683,11 @@ const char* shampoo_strerror(int code) {
 }
 
 void shampoo_destroy(shampoo_ctx* ctx) { delete ctx; }
+
+int shampoo_debug_inject_timeout(void) {
+  dash::arm_load_fault();
+  return SHAMPOO_OK;
+}
 
 }  // extern "C"
 

@@ -8,11 +8,11 @@
 // accumulators (tcgen05, kind::f16), which gives about fp32 accuracy at the
 // fp16 tensor-core rate.
 //
-// Both operands are read K-major: problem p computes
-//     out_p = s_p * (alpha * A_p Bm_p^T + beta * Cin_p + gamma * I)
-// where A_p and Bm_p are row-major matrices of the operand stacks.  A product
-// A * B is therefore formed from a stored B^T (the library keeps transposed
-// copies where an iterate is not symmetric).  A launch carries one or two
+// Problem p computes
+//     out_p = s_p * (alpha * A_p op(B_p) + beta * Cin_p + gamma * I)
+// where A_p is a row-major matrix of the A stack (read K-major) and op(B_p)
+// is B_p (b_mn = 1: the stored row-major B is read MN-major, giving A B) or
+// B_p^T (b_mn = 0: read K-major, giving A B^T).  A launch carries one or two
 // "ops" (groups of problems) with their own operand stacks and epilogues.
 // With sym = 1 only upper-triangle tiles are computed and each off-diagonal
 // tile is also written mirrored (for results that are symmetric by
@@ -43,7 +43,8 @@ struct Idx {
 
 struct GemmOp {
   int nprob;
-  Idx a, b;                  // operand matrices in this op's A / Bm stacks
+  Idx a, b;                  // operand matrices in this op's A / B stacks
+  int b_mn;                  // 1: out = A B ; 0: out = A B^T
   float alpha, beta, gamma;
   const float* scale;        // per-problem multiplier s_p (nullptr: 1)
   Idx scale_i;
@@ -69,6 +70,8 @@ struct GemmArgs {
   int B;      // matrix size; multiple of 128
   int sym;    // 1: symmetric outputs (upper-triangle tiles + mirrored writes)
   int nops;   // 1 or 2
+  int flush;  // 64-wide K slabs per hi*hi register flush (0: library default)
+  int skip_loads;  // test hook: the producer issues no loads (bounded waits expire)
   GemmOp op[2];
   unsigned* status;  // device status word (non-finite / timeout bits)
 };
@@ -85,5 +88,9 @@ struct OpBuffers {
 // Launch one batched GEMM (args.nops ops).  Returns cudaSuccess or the
 // launch / encode error.
 cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaStream_t stream);
+
+// Arm a one-shot test fault: the next GEMM launch withholds its operand loads,
+// so its waits run into their time limit and it reports a timeout.
+void arm_load_fault();
 
 }  // namespace dash

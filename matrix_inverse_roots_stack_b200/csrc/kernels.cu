@@ -13,111 +13,151 @@ namespace {
 // computes 128 rows of W = A V (32 columns) for one factor, streaming A in
 // 128 x 32 slabs through shared memory.
 
-constexpr int kPiRows = 128;
-constexpr int kPiK = 32;
+constexpr int kPiRows = 128;  // rows of W per CTA
+constexpr int kPiK = 32;      // K chunk per shared-memory stage
+constexpr int kPiPad = 4;     // padding of the transposed A tile (bank spread)
+
+// One chunk of the factor (128 rows x 32 k) and of V (32 k x 32 starts),
+// held in registers between global loads and shared-memory stores.
+struct PiChunk {
+  float4 a[4];
+  float4 v;
+};
+
+__device__ __forceinline__ PiChunk pi_load(const float* __restrict__ Fm, const float* __restrict__ Vsrc,
+                                           const float* inv, int B, int b, int r0, int k0, float eps, int t) {
+  PiChunk c;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {  // 1024 float4 of A: row = f / 8, k quad = f % 8
+    const int f = t + 256 * j;
+    const int rr = r0 + f / 8, kk = k0 + 4 * (f % 8);
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (rr < b) {
+      if (kk + 3 < b) {
+        x = *reinterpret_cast<const float4*>(Fm + static_cast<size_t>(rr) * B + kk);
+      } else {
+        float tmp[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tmp[e] = (kk + e < b) ? Fm[static_cast<size_t>(rr) * B + kk + e] : 0.0f;
+        x = make_float4(tmp[0], tmp[1], tmp[2], tmp[3]);
+      }
+      if (rr >= kk && rr < kk + 4) {  // regulariser on the diagonal
+        if (rr == kk) x.x += eps;
+        if (rr == kk + 1) x.y += eps;
+        if (rr == kk + 2) x.z += eps;
+        if (rr == kk + 3) x.w += eps;
+      }
+    }
+    c.a[j] = x;
+  }
+  {  // 256 float4 of V: k = t / 8, columns 4 * (t % 8)
+    const int kk = k0 + t / 8, cc = 4 * (t % 8);
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (kk < b) {
+      x = *reinterpret_cast<const float4*>(Vsrc + static_cast<size_t>(kk) * kPiStarts + cc);
+      x.x *= inv[cc];
+      x.y *= inv[cc + 1];
+      x.z *= inv[cc + 2];
+      x.w *= inv[cc + 3];
+    }
+    c.v = x;
+  }
+  return c;
+}
+
+__device__ __forceinline__ void pi_store(const PiChunk& c, float (*As)[kPiRows + kPiPad], float (*Vs)[kPiStarts],
+                                         int t) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int f = t + 256 * j;
+    const int rr = f / 8, kq = 4 * (f % 8);
+    As[kq][rr] = c.a[j].x;
+    As[kq + 1][rr] = c.a[j].y;
+    As[kq + 2][rr] = c.a[j].z;
+    As[kq + 3][rr] = c.a[j].w;
+  }
+  *reinterpret_cast<float4*>(&Vs[t / 8][4 * (t % 8)]) = c.v;
+}
 
 __global__ void __launch_bounds__(256) pi_iter_kernel(const float* __restrict__ F, int B, float eps,
                                                       const int* __restrict__ fsize, const float* __restrict__ v0,
                                                       const float* __restrict__ Wprev,
                                                       const float* __restrict__ sprev, float* __restrict__ Wnext,
                                                       float* __restrict__ snext) {
-  __shared__ float As[kPiRows][kPiK + 1];
+  __shared__ __align__(16) float As[kPiK][kPiRows + kPiPad];  // transposed: As[k][row]
   __shared__ __align__(16) float Vs[kPiK][kPiStarts];
   __shared__ float inv[kPiStarts];
-  __shared__ float red[8][3][kPiStarts];
+  __shared__ float red[3][32][kPiStarts + 1];
 
   const int f = blockIdx.y;
   const int r0 = blockIdx.x * kPiRows;
   const int b = fsize ? fsize[f] : B;
   const int t = threadIdx.x;
-  const int warp = t >> 5, lane = t & 31;
+  const int ty = t >> 3, tx = t & 7;  // rows 4ty..4ty+3, columns 4tx..4tx+3
   if (t < kPiStarts) {
-    float n2 = Wprev ? sprev[static_cast<size_t>(f) * 3 * kPiStarts + t] : 1.0f;
+    const float n2 = Wprev ? sprev[static_cast<size_t>(f) * 3 * kPiStarts + t] : 1.0f;
     inv[t] = Wprev ? (n2 > 0.0f ? rsqrtf(n2) : 0.0f) : 1.0f;
   }
   __syncthreads();
 
   const float* Fm = F + static_cast<size_t>(f) * B * B;
   const float* Vsrc = Wprev ? Wprev + static_cast<size_t>(f) * B * kPiStarts : v0;
-  const int row = t >> 1;
-  const int cb = (t & 1) * 16;
-  float acc[16];
+  float acc[4][4];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
 
   if (r0 < b) {
+    PiChunk nxt = pi_load(Fm, Vsrc, inv, B, b, r0, 0, eps, t);
     for (int k0 = 0; k0 < b; k0 += kPiK) {
-#pragma unroll
-      for (int i = 0; i < (kPiRows * kPiK) / 256; ++i) {
-        const int idx = i * 256 + t;
-        const int rr = idx / kPiK, kk = idx % kPiK;
-        const int gr = r0 + rr, gk = k0 + kk;
-        float a = 0.0f;
-        if (gr < b && gk < b) a = Fm[static_cast<size_t>(gr) * B + gk] + (gr == gk ? eps : 0.0f);
-        As[rr][kk] = a;
-      }
-#pragma unroll
-      for (int i = 0; i < (kPiK * kPiStarts) / 256; ++i) {
-        const int idx = i * 256 + t;
-        const int kk = idx / kPiStarts, c = idx % kPiStarts;
-        const int gk = k0 + kk;
-        Vs[kk][c] = gk < b ? Vsrc[static_cast<size_t>(gk) * kPiStarts + c] * inv[c] : 0.0f;
-      }
       __syncthreads();
+      pi_store(nxt, As, Vs, t);
+      __syncthreads();
+      if (k0 + kPiK < b) nxt = pi_load(Fm, Vsrc, inv, B, b, r0, k0 + kPiK, eps, t);
 #pragma unroll 8
       for (int kk = 0; kk < kPiK; ++kk) {
-        const float a = As[row][kk];
-        const float4* v4 = reinterpret_cast<const float4*>(&Vs[kk][cb]);
+        const float4 a = *reinterpret_cast<const float4*>(&As[kk][4 * ty]);
+        const float4 v = *reinterpret_cast<const float4*>(&Vs[kk][4 * tx]);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+        const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 v = v4[q];
-          acc[4 * q] += a * v.x;
-          acc[4 * q + 1] += a * v.y;
-          acc[4 * q + 2] += a * v.z;
-          acc[4 * q + 3] += a * v.w;
-        }
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] += av[i] * vv[j];
       }
-      __syncthreads();
     }
   }
 
-  const int gr = r0 + row;
-  float* Wo = Wnext + static_cast<size_t>(f) * B * kPiStarts + static_cast<size_t>(gr) * kPiStarts + cb;
+  // write W rows and accumulate the column statistics of this CTA's rows
+  float w2[4] = {0.f, 0.f, 0.f, 0.f}, vw[4] = {0.f, 0.f, 0.f, 0.f}, v2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int j = 0; j < 16; ++j) Wo[j] = acc[j];
-
-  // column statistics of this CTA's rows
-  float w2[16], vw[16], v2[16];
+  for (int i = 0; i < 4; ++i) {
+    const int gr = r0 + 4 * ty + i;
+    float* Wo = Wnext + static_cast<size_t>(f) * B * kPiStarts + static_cast<size_t>(gr) * kPiStarts + 4 * tx;
+    *reinterpret_cast<float4*>(Wo) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    float4 vr = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (gr < b) vr = *reinterpret_cast<const float4*>(Vsrc + static_cast<size_t>(gr) * kPiStarts + 4 * tx);
+    const float vv[4] = {vr.x * inv[4 * tx], vr.y * inv[4 * tx + 1], vr.z * inv[4 * tx + 2], vr.w * inv[4 * tx + 3]};
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float v = gr < b ? Vsrc[static_cast<size_t>(gr) * kPiStarts + cb + j] * inv[cb + j] : 0.0f;
-    w2[j] = acc[j] * acc[j];
-    vw[j] = v * acc[j];
-    v2[j] = v * v;
-  }
-#pragma unroll
-  for (int o = 2; o < 32; o <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      w2[j] += __shfl_xor_sync(0xffffffffu, w2[j], o);
-      vw[j] += __shfl_xor_sync(0xffffffffu, vw[j], o);
-      v2[j] += __shfl_xor_sync(0xffffffffu, v2[j], o);
+    for (int j = 0; j < 4; ++j) {
+      w2[j] += acc[i][j] * acc[i][j];
+      vw[j] += vv[j] * acc[i][j];
+      v2[j] += vv[j] * vv[j];
     }
   }
-  if (lane < 2) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      red[warp][0][cb + j] = w2[j];
-      red[warp][1][cb + j] = vw[j];
-      red[warp][2][cb + j] = v2[j];
-    }
+  for (int j = 0; j < 4; ++j) {
+    red[0][ty][4 * tx + j] = w2[j];
+    red[1][ty][4 * tx + j] = vw[j];
+    red[2][ty][4 * tx + j] = v2[j];
   }
   __syncthreads();
   if (t < 3 * kPiStarts) {
     const int q = t / kPiStarts, c = t % kPiStarts;
     float s = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) s += red[w][q][c];
+#pragma unroll 8
+    for (int y = 0; y < 32; ++y) s += red[q][y][c];
     if (s != 0.0f) atomicAdd(&snext[static_cast<size_t>(f) * 3 * kPiStarts + q * kPiStarts + c], s);
   }
 }
@@ -158,84 +198,54 @@ __device__ __forceinline__ void load_split4(const __half* base, size_t BB, size_
   for (int e = 0; e < 4; ++e) x[e] = join_f16(h[e], l[e]);
 }
 
-// Newton-DB prologues.  grid (B/32, B/32, nf), block (32, 8): each CTA owns a
-// 32 x 32 tile, writes its outputs in place and, through shared memory, the
-// transposed copies the K-major GEMM needs (exact transposes, so the stage-2
-// iterates, which are not exactly symmetric, keep consistent copies).
+// Newton-DB prologues (element-wise; grid (B*B/1024, nf), 256 threads, 4
+// consecutive elements per thread).
 
-__device__ __forceinline__ void put_split(__half* base, size_t BB, size_t idx, float x) {
-  __half h, l;
-  split_f16(x, h, l);
-  base[idx] = h;
-  base[BB + idx] = l;
-}
-
-__global__ void ndb_init_kernel(const float* __restrict__ F, int B, float eps, const int* __restrict__ fsize,
-                                const float* __restrict__ lam, float zs, __half* __restrict__ Y0,
-                                __half* __restrict__ D0, __half* __restrict__ D0t, __half* __restrict__ Z1,
-                                __half* __restrict__ Z1t, float* __restrict__ xscale) {
-  __shared__ float td[32][33], tz[32][33];
-  const int f = blockIdx.z;
+__global__ void __launch_bounds__(256) ndb_init_kernel(const float* __restrict__ F, int B, float eps,
+                                                       const int* __restrict__ fsize,
+                                                       const float* __restrict__ lam, float zs,
+                                                       __half* __restrict__ Y0, __half* __restrict__ D0,
+                                                       __half* __restrict__ Z1, float* __restrict__ xscale) {
+  const int f = blockIdx.y;
   const size_t BB = static_cast<size_t>(B) * B;
-  const int tr = blockIdx.y * 32, tc = blockIdx.x * 32;
+  const size_t idx = (static_cast<size_t>(blockIdx.x) * 256 + threadIdx.x) * 4;
   const int b = fsize ? fsize[f] : B;
   const float c = 0.5f / lam[f];
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) xscale[f] = sqrtf(sqrtf(c)) * zs;
-  const float* Fm = F + f * BB;
-  const size_t off = static_cast<size_t>(f) * 2 * BB;
+  if (idx == 0) xscale[f] = sqrtf(sqrtf(c)) * zs;
+  const int r = static_cast<int>(idx / B), col = static_cast<int>(idx % B);
+  const float4 a4 = *reinterpret_cast<const float4*>(F + f * BB + idx);
+  const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+  float y[4], d[4], z[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = tr + threadIdx.y + 8 * i, col = tc + threadIdx.x;
-    const float id = (r == col) ? 1.0f : 0.0f;
-    const float a = (r < b && col < b) ? c * (Fm[static_cast<size_t>(r) * B + col] + id * eps) : id;
-    const float d = 0.5f * (id - a);
-    const float z = (id + d) / zs;
-    const size_t e = static_cast<size_t>(r) * B + col;
-    put_split(Y0 + off, BB, e, a);
-    put_split(D0 + off, BB, e, d);
-    put_split(Z1 + off, BB, e, z);
-    td[threadIdx.y + 8 * i][threadIdx.x] = d;
-    tz[threadIdx.y + 8 * i][threadIdx.x] = z;
+  for (int e = 0; e < 4; ++e) {
+    const int cc = col + e;
+    const float id = (r == cc) ? 1.0f : 0.0f;
+    const float a = (r < b && cc < b) ? c * (av[e] + id * eps) : id;
+    y[e] = a;
+    d[e] = 0.5f * (id - a);
+    z[e] = (id + d[e]) / zs;
   }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = tc + threadIdx.y + 8 * i, col = tr + threadIdx.x;
-    const size_t e = static_cast<size_t>(r) * B + col;
-    put_split(D0t + off, BB, e, td[threadIdx.x][threadIdx.y + 8 * i]);
-    put_split(Z1t + off, BB, e, tz[threadIdx.x][threadIdx.y + 8 * i]);
-  }
+  store_split4(Y0 + 2 * f * BB, BB, idx, y);
+  store_split4(D0 + 2 * f * BB, BB, idx, d);
+  store_split4(Z1 + 2 * f * BB, BB, idx, z);
 }
 
-__global__ void ndb_stage2_init_kernel(const __half* __restrict__ Y, int B, float zs, __half* __restrict__ D0,
-                                       __half* __restrict__ D0t, __half* __restrict__ Z1,
-                                       __half* __restrict__ Z1t) {
-  __shared__ float td[32][33], tz[32][33];
-  const int f = blockIdx.z;
+__global__ void __launch_bounds__(256) ndb_stage2_init_kernel(const __half* __restrict__ Y, int B, float zs,
+                                                              __half* __restrict__ D0, __half* __restrict__ Z1) {
+  const int f = blockIdx.y;
   const size_t BB = static_cast<size_t>(B) * B;
-  const int tr = blockIdx.y * 32, tc = blockIdx.x * 32;
-  const size_t off = static_cast<size_t>(f) * 2 * BB;
+  const size_t idx = (static_cast<size_t>(blockIdx.x) * 256 + threadIdx.x) * 4;
+  const int r = static_cast<int>(idx / B), col = static_cast<int>(idx % B);
+  float y[4], d[4], z[4];
+  load_split4(Y + 2 * f * BB, BB, idx, y);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = tr + threadIdx.y + 8 * i, col = tc + threadIdx.x;
-    const size_t e = static_cast<size_t>(r) * B + col;
-    const float id = (r == col) ? 1.0f : 0.0f;
-    const float y = join_f16(Y[off + e], Y[off + BB + e]);
-    const float d = 0.5f * (id - y);
-    const float z = (id + d) / zs;
-    put_split(D0 + off, BB, e, d);
-    put_split(Z1 + off, BB, e, z);
-    td[threadIdx.y + 8 * i][threadIdx.x] = d;
-    tz[threadIdx.y + 8 * i][threadIdx.x] = z;
+  for (int e = 0; e < 4; ++e) {
+    const float id = (r == col + e) ? 1.0f : 0.0f;
+    d[e] = 0.5f * (id - y[e]);
+    z[e] = (id + d[e]) / zs;
   }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = tc + threadIdx.y + 8 * i, col = tr + threadIdx.x;
-    const size_t e = static_cast<size_t>(r) * B + col;
-    put_split(D0t + off, BB, e, td[threadIdx.x][threadIdx.y + 8 * i]);
-    put_split(Z1t + off, BB, e, tz[threadIdx.x][threadIdx.y + 8 * i]);
-  }
+  store_split4(D0 + 2 * f * BB, BB, idx, d);
+  store_split4(Z1 + 2 * f * BB, BB, idx, z);
 }
 
 __global__ void __launch_bounds__(256) scale_split_kernel(const __half* __restrict__ Z, int B,
@@ -449,17 +459,15 @@ void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* l
 }
 
 void launch_ndb_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, float zs,
-                     __half* Y0, __half* D0, __half* D0t, __half* Z1, __half* Z1t, float* xscale,
-                     cudaStream_t st) {
-  dim3 grid(B / 32, B / 32, nf);
-  ndb_init_kernel<<<grid, dim3(32, 8), 0, st>>>(F, B, eps, fsize, lambda, zs, Y0, D0, D0t, Z1, Z1t, xscale);
+                     __half* Y0, __half* D0, __half* Z1, float* xscale, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(static_cast<size_t>(B) * B / 1024), nf);
+  ndb_init_kernel<<<grid, 256, 0, st>>>(F, B, eps, fsize, lambda, zs, Y0, D0, Z1, xscale);
   prof_count_launch();
 }
 
-void launch_ndb_stage2_init(const __half* Y, int nf, int B, float zs, __half* D0, __half* D0t, __half* Z1,
-                            __half* Z1t, cudaStream_t st) {
-  dim3 grid(B / 32, B / 32, nf);
-  ndb_stage2_init_kernel<<<grid, dim3(32, 8), 0, st>>>(Y, B, zs, D0, D0t, Z1, Z1t);
+void launch_ndb_stage2_init(const __half* Y, int nf, int B, float zs, __half* D0, __half* Z1, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(static_cast<size_t>(B) * B / 1024), nf);
+  ndb_stage2_init_kernel<<<grid, 256, 0, st>>>(Y, B, zs, D0, Z1);
   prof_count_launch();
 }
 

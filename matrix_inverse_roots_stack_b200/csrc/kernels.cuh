@@ -40,15 +40,12 @@ void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* l
 
 // Newton-DB stage-1 prologue: c = 1/(2 lambda); Y0 = c (F + eps I) (padding:
 // identity); D0 = (I - Y0)/2; Zhat1 = (I + D0)/zs; xscale = c^(1/4) zs.
-// D0 and Zhat1 are also written transposed (D0t, Z1t).
 void launch_ndb_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, float zs,
-                     __half* Y0, __half* D0, __half* D0t, __half* Z1, __half* Z1t, float* xscale,
-                     cudaStream_t st);
+                     __half* Y0, __half* D0, __half* Z1, float* xscale, cudaStream_t st);
 
 // Newton-DB stage-2 prologue from the split Y of stage 1:
-// D0 = (I - Y)/2; Zhat1 = (I + D0)/zs; both also written transposed.
-void launch_ndb_stage2_init(const __half* Y, int nf, int B, float zs, __half* D0, __half* D0t, __half* Z1,
-                            __half* Z1t, cudaStream_t st);
+// D0 = (I - Y)/2; Zhat1 = (I + D0)/zs.
+void launch_ndb_stage2_init(const __half* Y, int nf, int B, float zs, __half* D0, __half* Z1, cudaStream_t st);
 
 // out = xscale_f * Zhat (split in; fp32 and/or split out); used when a stage
 // has a single iteration.

@@ -25,16 +25,17 @@ EncodeTiledFn get_encoder() {
 
 }  // namespace
 
-cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat) {
+cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat, int box_rows) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return cudaErrorInvalidValue;
-  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || B % 128 != 0 || nmat < 1)
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || B % 128 != 0 || nmat < 1 || box_rows < 1 ||
+      box_rows > 256)
     return cudaErrorInvalidValue;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(B), static_cast<cuuint64_t>(B),
                         static_cast<cuuint64_t>(2) * static_cast<cuuint64_t>(nmat)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(B) * 2u,
                            static_cast<cuuint64_t>(B) * static_cast<cuuint64_t>(B) * 2u};
-  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estride[3] = {1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -10,8 +10,8 @@
 namespace dash {
 
 // Encode a 3-D tiled map over a split stack: dims {B (columns, innermost),
-// B (rows), 2 * nmat (matrix * 2 + plane)} of fp16, box {64, 128, 1},
+// B (rows), 2 * nmat (matrix * 2 + plane)} of fp16, box {64, box_rows, 1},
 // 128-byte swizzle.  Returns cudaSuccess or cudaErrorInvalidValue.
-cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat);
+cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat, int box_rows = 128);
 
 }  // namespace dash

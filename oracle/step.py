@@ -185,3 +185,22 @@ def shampoo_step(thetas, grads, state, hp, V0, lam_override=None):
         P_out.append(P)
     info = {"lam": lam_out, "graft": graft_out, "U": U_out, "P": P_out}
     return new_thetas, {"params": new_params, "t": t}, info
+
+
+def first_step_block_update(Gb, Pb, hp, lam_L, lam_R):
+    """Delta theta of one block on the first step, from its gradient block.
+
+    Same arithmetic as :func:`shampoo_step` restricted to one block (factors
+    start at init_scale*I; P is that block of the Adam direction), so that
+    sampled blocks of a large parameter set can be checked one by one.
+    Returns (delta, U, s).
+    """
+    Gb = np.asarray(Gb, dtype=np.float64)
+    br, bc = Gb.shape
+    L, R = factor_ema(hp.init_scale * np.eye(br), hp.init_scale * np.eye(bc), Gb, hp.beta)
+    XL, _ = inverse_fourth_root(L + hp.eps * np.eye(br), None, hp, lam_L)
+    XR, _ = inverse_fourth_root(R + hp.eps * np.eye(bc), None, hp, lam_R)
+    U = XL @ Gb @ XR
+    s = graft_scale(Pb, U)
+    return -hp.lr * s * U, U, s
+

@@ -137,3 +137,18 @@ def test_standalone_workload_full_size(torch):
     assert rc == 0
     errs = [rel(X[i], r) for i, r in enumerate(cheb_level2(A, 0.0, lam, 16, 1e-3))]
     assert max(errs) < ROOT_TOL, max(errs)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(torch):
+    # a GEMM launch that never receives its operand tiles: every wait gives up
+    # after its limit, the status word says TIMEOUT, and the next call works
+    from matrix_inverse_roots_stack_b200 import binding as bd
+    A = workloads.spd_stack_geometric(1, 128, 10.0, seed=12)
+    lib = bd.load()
+    assert lib.shampoo_debug_inject_timeout() == 0
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=2, iters2=2)
+    assert rc == bd.SHAMPOO_ETIMEOUT
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=6, iters2=6)
+    assert rc == 0
+    ref = roots.ndb_inv4root_spectral(A[0].astype(np.float64), lam[0], 6, 6)
+    assert rel(X[0], ref) < ROOT_TOL

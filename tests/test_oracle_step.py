@@ -152,3 +152,15 @@ def test_converged_truncated_step_matches_exact_step():
         out[level] = new[0]
     assert rel(out[2], out[1]) < 1e-9
     assert rel(out[3], out[2]) < 1e-9
+
+
+def test_first_step_block_update_matches_full_step():
+    G = workloads.gaussian_gradients([(40, 24)], std=0.1, seed=11)[0].astype(np.float64)
+    hp = step.HParams(block_size=16, ndb_iters1=9, ndb_iters2=9)
+    V0 = workloads.pi_start_vectors(16, 32, seed=0)
+    th0 = np.zeros(G.shape)
+    new, _, info = step.shampoo_step([th0], [G], step.init_state([G.shape], hp), hp, V0)
+    for k, (r0, r1, c0, c1) in enumerate(step.block_grid(40, 24, 16)):
+        d, _, s = step.first_step_block_update(G[r0:r1, c0:c1], info["P"][0][r0:r1, c0:c1], hp,
+                                               info["lam"][2 * k], info["lam"][2 * k + 1])
+        assert rel(d, new[0][r0:r1, c0:c1]) < 1e-13 and s == pytest.approx(info["graft"][k], rel=1e-13)

@@ -62,8 +62,10 @@ def test_static_scratch_matches_workspace_entry_point(torch):
 def test_static_scratch_rejects_oversized_problem(torch):
     from matrix_inverse_roots_stack_b200 import binding as bd
     lib = bd.load()
-    n, B = 2, 1024  # needs more than the 64 MiB scratch
-    assert lib.shampoo_inv_root_workspace_bytes(n, B, 0) > bd.STATIC_SCRATCH_BYTES
+    B = 1024
+    n = 1
+    while lib.shampoo_inv_root_workspace_bytes(n, B, 0) <= bd.STATIC_SCRATCH_BYTES:
+        n += 1  # smallest stack that does not fit the 64 MiB scratch
     At = torch.zeros((n, B, B), dtype=torch.float32, device="cuda")
     vt = torch.zeros((B, 32), dtype=torch.float32, device="cuda")
     rc, _, _ = call_static(torch, lib, At, vt, 4, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))

@@ -2,22 +2,24 @@
 // warp-specialised.
 //
 // Each CTA (one per SM) walks a static round-robin list of 128 x 128 output
-// tiles of all problems of the launch.  Roles (192 threads):
+// tiles of all problems of the launch.  Roles (320 threads):
 //   warp 0, one lane   TMA producer: streams the A hi/lo and B hi/lo tiles of
 //                      each 64-wide K slab into a 3-stage shared-memory ring
 //                      (A always K-major; B K-major, or MN-major as two
 //                      64-column boxes when the op multiplies by B itself);
 //   warp 1, one lane   MMA issuer;
-//   warps 2-5          epilogue; warp w reads tensor-memory lanes 32*(w%4)..
+//   warps 2-9          epilogue; warp w reads tensor-memory lanes 32*(w%4)..
+//                      and columns 64*((w-2)/4).. of each accumulator, so
+//                      every thread owns 64 columns of one output row.
 // Tensor memory (512 columns): a ring of three 128-column hi*hi accumulators
 // and one 128-column lo accumulator.
 //
-// The tensor core's fp32 accumulation truncates (about -0.5 ulp per MMA, so
-// the bias grows linearly with K).  The hi*hi products, which carry the
+// The tensor core's fp32 accumulation truncates (the bias grows linearly
+// with the number of MMAs accumulated).  The hi*hi products, which carry the
 // result's magnitude, are therefore accumulated in tensor memory over one
-// flush segment only (args.flush 64-wide slabs, default one) and then added
-// with round-to-nearest into fp32 registers of the epilogue warps, while the
-// MMA warp fills the next ring buffer.  The hi*lo + lo*hi products enter the
+// flush segment only (args.flush K=16 MMAs, default one) and then added
+// with round-to-nearest into fp32 registers of the epilogue warps (packed
+// f32x2 adds), while the MMA warp fills the next ring buffer.  The hi*lo + lo*hi products enter the
 // result scaled by 2^-11 and stay in tensor memory for the whole K range;
 // they are read into the registers as soon as a tile's last MMA retires, so
 // the next tile can start while the epilogue writes the previous one out.
@@ -36,12 +38,20 @@ constexpr int kKBlk = 64;                          // fp16 elements per 128-byte
 constexpr int kStages = 3;
 constexpr int kTileBytes = kTile * kKBlk * 2;      // 16 KB
 constexpr int kStageBytes = 4 * kTileBytes;        // A hi, A lo, B hi, B lo
-constexpr int kThreads = 192;
+#ifndef DASH_EPI_WARPS
+#define DASH_EPI_WARPS 8
+#endif
 constexpr int kEpiWarp0 = 2;
+constexpr int kEpiWarps = DASH_EPI_WARPS;          // 4 or 8
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr int kCols = kTile * 4 / kEpiWarps;       // accumulator columns per epilogue thread
 constexpr int kRing = 3;                           // hi*hi accumulators
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColLO = kRing * 128;           // lo accumulator
-constexpr int kDefaultFlush = 1;                   // slabs per hi*hi flush
+#ifndef DASH_FLUSH_MMAS
+#define DASH_FLUSH_MMAS 1
+#endif
+constexpr int kDefaultFlush = DASH_FLUSH_MMAS;     // K=16 MMAs per hi*hi flush
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
@@ -166,6 +176,8 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// FL: K=16 MMAs per hi*hi flush segment (1, 2 or 4), or 0 for one segment per tile.
+template <int FL>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_split_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                       const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -180,8 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt = args.B / kTile;
   const int tpp = args.sym ? nt * (nt + 1) / 2 : nt * nt;
   const int nk = args.B / kKBlk;
-  const int fl = args.flush;  // slabs per flush segment (divides nk)
-  const int nseg = nk / fl;
+  const int nseg = FL == 0 ? 1 : nk * (kKBlk / 16) / FL;  // flush segments per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -190,10 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < kRing; ++b) {
       mbar_init(&bars->hh_full[b], 1);
-      mbar_init(&bars->hh_empty[b], 4);
+      mbar_init(&bars->hh_empty[b], kEpiWarps);
     }
     mbar_init(&bars->lo_full, 1);
-    mbar_init(&bars->lo_empty, 4);
+    mbar_init(&bars->lo_empty, kEpiWarps);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -214,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      uint32_t sc = 0;
+      uint32_t sc = 0, s = 0, epar = 1;  // loads issued, stage, parity of the stage's next release
       bool stop = args.skip_loads != 0;
       for (long long t = blockIdx.x; t < total && !stop; t += gridDim.x) {
         int op, p, ti, tj;
@@ -224,8 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* ta = op ? &tmA1 : &tmA0;
         const CUtensorMap* tb = op ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb, ++sc) {
-          const uint32_t s = sc % kStages, ph = (sc / kStages) & 1u;
-          if (sc >= kStages && !mbar_wait(&bars->empty[s], ph ^ 1u, abort_flag)) {
+          if (!mbar_wait(&bars->empty[s], epar, abort_flag)) {  // fresh barriers pass on parity 1
             fail_timeout(abort_flag, args.status);
             stop = true;
             break;
@@ -245,6 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(st + 2 * kTileBytes, tb, &bars->full[s], kb * kKBlk, tj * kTile, 2 * bm);
             tma_load_3d(st + 3 * kTileBytes, tb, &bars->full[s], kb * kKBlk, tj * kTile, 2 * bm + 1);
           }
+          if (++s == kStages) {
+            s = 0;
+            epar ^= 1u;
+          }
         }
       }
       if (*abort_flag) {  // let this CTA's own copies land before it can exit
@@ -255,54 +269,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // One thread issues every MMA of the CTA, so this loop is kept to a few
+    // scalar instructions per K=16 step: descriptors are a base plus
+    // compile-time offsets, ring positions advance without division, and
+    // the release barriers start out passable (parity 1 on a fresh barrier).
     if (lane == 0) {
-      uint32_t sc = 0, gk = 0;  // gk counts flush segments
-      bool stop = false;
-      int i = 0;
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t kd0 = sw128_kmajor_desc(sbase), md0 = sw128_mnmajor_desc(sbase);
+      constexpr uint32_t kTileD = kTileBytes >> 4;  // descriptor address units
+      uint32_t s = 0, fpar = 0;                     // stage, parity of its next fill
+      uint32_t hb = 0, hpar = (1u << kRing) - 1u;   // hh buffer, parity bits of the next release per buffer
+      uint32_t lpar = 1u;                           // parity of the lo accumulator's next release
+      bool ok = true;
       const uint32_t lo_t = tbase + kColLO;
-      for (long long t = blockIdx.x; t < total && !stop; t += gridDim.x, ++i) {
+      for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
         int op, p, ti, tj;
         decode(args, tpp, nt, t, op, p, ti, tj);
         const bool bmn = args.op[op].b_mn != 0;
         const uint32_t idesc = f16_idesc(128, 128) | (bmn ? (1u << 16) : 0u);
-        if (i >= 1 && !mbar_wait(&bars->lo_empty, (i - 1) & 1u, abort_flag)) {
-          fail_timeout(abort_flag, args.status);
-          break;
-        }
-        for (int kb = 0; kb < nk; ++kb, ++sc) {
-          const uint32_t s = sc % kStages, ph = (sc / kStages) & 1u;
-          const uint32_t hb = gk % kRing;
-          const bool seg_first = (kb % fl) == 0, seg_last = (kb % fl) == fl - 1;
-          if (!mbar_wait(&bars->full[s], ph, abort_flag) ||
-              (seg_first && gk >= kRing &&
-               !mbar_wait(&bars->hh_empty[hb], ((gk / kRing) & 1u) ^ 1u, abort_flag))) {
-            fail_timeout(abort_flag, args.status);
-            stop = true;
-            break;
-          }
+        const uint64_t bd0 = (bmn ? md0 : kd0) + 2 * kTileD;
+        const uint32_t bstep = bmn ? (2048u >> 4) : (32u >> 4);
+        ok = mbar_wait(&bars->lo_empty, lpar, abort_flag);
+        lpar ^= 1u;
+        if (!ok) break;
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb) {
+          ok = mbar_wait(&bars->full[s], fpar, abort_flag);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t hh_t = tbase + hb * 128u;
-          const uint32_t st = smem_u32(smem + s * kStageBytes);
+          const uint32_t so = s * (kStageBytes >> 4);
+          const uint64_t ah = kd0 + so, al = ah + kTileD, bh = bd0 + so, bl = bh + kTileD;
 #pragma unroll
           for (int kk = 0; kk < kKBlk / 16; ++kk) {
-            const uint64_t ah = sw128_kmajor_desc(st + kk * 32);
-            const uint64_t al = sw128_kmajor_desc(st + kTileBytes + kk * 32);
-            const uint64_t bh = bmn ? sw128_mnmajor_desc(st + 2 * kTileBytes + kk * 2048)
-                                    : sw128_kmajor_desc(st + 2 * kTileBytes + kk * 32);
-            const uint64_t bl = bmn ? sw128_mnmajor_desc(st + 3 * kTileBytes + kk * 2048)
-                                    : sw128_kmajor_desc(st + 3 * kTileBytes + kk * 32);
-            mma_f16_ss(hh_t, ah, bh, idesc, (seg_first && kk == 0) ? 0u : 1u);
-            mma_f16_ss(lo_t, ah, bl, idesc, (kb | kk) != 0 ? 1u : 0u);
-            mma_f16_ss(lo_t, al, bh, idesc, 1u);
+            const bool seg_start = FL == 0 ? (kb == 0 && kk == 0) : (kk % FL) == 0;
+            const bool seg_end = FL == 0 ? (kb == nk - 1 && kk == kKBlk / 16 - 1) : (kk % FL) == FL - 1;
+            if (seg_start) {
+              ok = mbar_wait(&bars->hh_empty[hb], (hpar >> hb) & 1u, abort_flag);
+              hpar ^= 1u << hb;
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint32_t ka = 2u * kk, kbo = bstep * kk;
+            mma_f16_ss(tbase + hb * 128u, ah + ka, bh + kbo, idesc, seg_start ? 0u : 1u);
+            mma_f16_ss(lo_t, ah + ka, bl + kbo, idesc, (kb == 0 && kk == 0) ? 0u : 1u);
+            mma_f16_ss(lo_t, al + ka, bh + kbo, idesc, 1u);
+            if (seg_end) {
+              mma_commit(&bars->hh_full[hb]);
+              hb = hb == kRing - 1 ? 0u : hb + 1u;
+            }
           }
+          if (!ok) break;
           mma_commit(&bars->empty[s]);
-          if (seg_last) {
-            mma_commit(&bars->hh_full[hb]);
-            ++gk;
-          }
           if (kb == nk - 1) mma_commit(&bars->lo_full);
+          if (++s == kStages) {
+            s = 0;
+            fpar ^= 1u;
+          }
         }
       }
+      if (!ok) fail_timeout(abort_flag, args.status);
       // all issued MMAs must retire before tensor memory is released
       mma_commit(&bars->drain);
       volatile int never = 0;
@@ -311,60 +336,76 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int half = (warp - kEpiWarp0) >> 2;
+    const uint32_t lane_off = (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(half * kCols);
     const size_t B = static_cast<size_t>(args.B);
     const size_t BB = B * B;
-    uint32_t gk = 0;
-    int i = 0;
-    for (long long t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+    uint32_t hb = 0, hpar = 0, lpar = 0;  // hh buffer and fill parities, lo fill parity
+    for (long long t = blockIdx.x; t < total; t += gridDim.x) {
       int op, p, ti, tj;
       decode(args, tpp, nt, t, op, p, ti, tj);
       const GemmOp& g = args.op[op];
-      {  // pull this tile's Cin rows into L2 while the mainloop runs
-        const size_t prow = static_cast<size_t>(ti * kTile + quad * 32 + lane) * B + static_cast<size_t>(tj) * kTile;
+      const int row = ti * kTile + quad * 32 + lane;
+      const int cbase = tj * kTile + half * kCols;
+      {  // pull this thread's Cin row segment into L2 while the mainloop runs
+        const size_t prow = static_cast<size_t>(row) * B + static_cast<size_t>(cbase);
         if (g.cin_split && !g.cin_trans) {
           const __half* cb = g.cin_split + static_cast<size_t>(at(g.cin_i, p)) * 2 * BB + prow;
           prefetch_l2(cb);
-          prefetch_l2(cb + 64);
           prefetch_l2(cb + BB);
-          prefetch_l2(cb + BB + 64);
         }
         if (g.cin_f32) {
           const float* cb = g.cin_f32 + static_cast<size_t>(at(g.cinf_i, p)) * BB + prow;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) prefetch_l2(cb + 32 * q);
+          prefetch_l2(cb);
+          prefetch_l2(cb + 32);
         }
       }
-      float S[kTile];
+      float S[kCols];
 #pragma unroll
-      for (int j = 0; j < kTile; ++j) S[j] = 0.0f;
+      for (int j = 0; j < kCols; ++j) S[j] = 0.0f;
 
       bool ok = true;
-      for (int sg = 0; sg < nseg; ++sg, ++gk) {
-        const uint32_t hb = gk % kRing;
-        if (!mbar_wait(&bars->hh_full[hb], (gk / kRing) & 1u, abort_flag)) {
+      for (int sg = 0; sg < nseg; ++sg) {
+        // epilogue warps sleep in the barrier while they wait, leaving the
+        // issue slots of their scheduler to the MMA and TMA threads
+        if (!mbar_wait_sleep(&bars->hh_full[hb], (hpar >> hb) & 1u, abort_flag)) {
           ok = false;
           break;
         }
+        hpar ^= 1u << hb;
         tc_fence_after();
         const uint32_t src = tbase + lane_off + hb * 128u;
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t r0[16], r1[16];
-          tmem_ld_32x32b_x16(src + c * 32, r0);
-          tmem_ld_32x32b_x16(src + c * 32 + 16, r1);
+        for (int c = 0; c < kCols / 64; ++c) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(src + 64 * c, r0);
+          tmem_ld_32x32b_x32(src + 64 * c + 32, r1);
           tmem_ld_wait();
+          if (c + 1 == kCols / 64) {  // registers hold the whole segment now
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->hh_empty[hb]);
+            hb = hb == kRing - 1 ? 0u : hb + 1u;
+          }
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            S[c * 32 + j] += __uint_as_float(r0[j]);
-            S[c * 32 + 16 + j] += __uint_as_float(r1[j]);
+          for (int j = 0; j < 32; j += 2) {
+#ifdef DASH_PLAIN_FADD
+            S[64 * c + j] += __uint_as_float(r0[j]);
+            S[64 * c + j + 1] += __uint_as_float(r0[j + 1]);
+            S[64 * c + 32 + j] += __uint_as_float(r1[j]);
+            S[64 * c + 32 + j + 1] += __uint_as_float(r1[j + 1]);
+#else
+            add_f32x2(S[64 * c + j], S[64 * c + j + 1], r0[j], r0[j + 1]);
+            add_f32x2(S[64 * c + 32 + j], S[64 * c + 32 + j + 1], r1[j], r1[j + 1]);
+#endif
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->hh_empty[hb]);
       }
-      if (!ok || !mbar_wait(&bars->lo_full, i & 1u, abort_flag)) {
+      if (ok) {
+        ok = mbar_wait_sleep(&bars->lo_full, lpar, abort_flag);
+        lpar ^= 1u;
+      }
+      if (!ok) {
         if (threadIdx.x == kEpiWarp0 * 32) fail_timeout(abort_flag, args.status);
         break;
       }
@@ -372,23 +413,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const uint32_t src = tbase + lane_off + kColLO;
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t r0[16], r1[16];
-          tmem_ld_32x32b_x16(src + c * 32, r0);
-          tmem_ld_32x32b_x16(src + c * 32 + 16, r1);
+        for (int h = 0; h < kCols / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(src + 32 * h, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            S[c * 32 + j] += __uint_as_float(r0[j]) * kLoUnscale;
-            S[c * 32 + 16 + j] += __uint_as_float(r1[j]) * kLoUnscale;
-          }
+          for (int j = 0; j < 32; ++j) S[32 * h + j] += __uint_as_float(r[j]) * kLoUnscale;
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->lo_empty);  // the next tile may start accumulating
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->lo_empty);  // the next tile may start accumulating
 
-      const int row = ti * kTile + quad * 32 + lane;
       const float s = g.scale ? g.scale[at(g.scale_i, p)] : 1.0f;
       const __half* cin = g.cin_split ? g.cin_split + static_cast<size_t>(at(g.cin_i, p)) * 2 * BB : nullptr;
       const float* cinf = g.cin_f32 ? g.cin_f32 + static_cast<size_t>(at(g.cinf_i, p)) * BB : nullptr;
@@ -403,17 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sumsq = 0.0f;
       const bool cin_rows = cin && !g.cin_trans;
       SplitChunk nxt;
-      if (cin_rows) nxt = ld_chunk(cin, BB, row * B + tj * kTile);
+      if (cin_rows) nxt = ld_chunk(cin, BB, row * B + cbase);
 
 #pragma unroll
-      for (int c = 0; c < kTile / 16; ++c) {
-        const int col0 = tj * kTile + c * 16;
-        float v[16];
+      for (int c = 0; c < kCols / 16; ++c) {
+        const int col0 = cbase + c * 16;
+        float* v = &S[c * 16];  // finished in place
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = g.alpha * S[c * 16 + j];
+        for (int j = 0; j < 16; ++j) v[j] *= g.alpha;
         if (cin_rows) {  // this chunk's Cin was loaded one chunk ahead
           const SplitChunk cur = nxt;
-          if (c + 1 < kTile / 16) nxt = ld_chunk(cin, BB, row * B + col0 + 16);
+          if (c + 1 < kCols / 16) nxt = ld_chunk(cin, BB, row * B + col0 + 16);
           float cj[16];
           join_chunk(cur, cj);
 #pragma unroll
@@ -520,11 +556,14 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
     e = encode_split_stack_map(&maps[2 * o + 1], b.b, a.B, b.b_nmat, a.op[o].b_mn ? 64 : 128);
     if (e != cudaSuccess) return e;
   }
-  const int nk = a.B / kKBlk;
+  const int nm = (a.B / kKBlk) * (kKBlk / 16);  // K=16 MMAs per tile
   if (a.flush <= 0) a.flush = kDefaultFlush;
-  if (a.flush > nk) a.flush = nk;
-  while (nk % a.flush) --a.flush;
-  cudaError_t e = cudaFuncSetAttribute(gemm_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmArgs,
+               const long long) = a.flush >= nm  ? gemm_split_kernel<0>
+                                  : a.flush >= 4 ? gemm_split_kernel<4>
+                                  : a.flush >= 2 ? gemm_split_kernel<2>
+                                                 : gemm_split_kernel<1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int nt = a.B / kTile;
   const long long tpp = a.sym ? nt * (nt + 1) / 2 : nt * nt;
@@ -534,7 +573,7 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   // useful flops: each computed 128 x 128 tile is one 2*128*128*B product
   const double flops = 2.0 * kTile * kTile * static_cast<double>(a.B) * static_cast<double>(total);
   const int slot = prof_begin(kProfGemm, stream, flops);
-  gemm_split_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

@@ -70,7 +70,7 @@ struct GemmArgs {
   int B;      // matrix size; multiple of 128
   int sym;    // 1: symmetric outputs (upper-triangle tiles + mirrored writes)
   int nops;   // 1 or 2
-  int flush;  // 64-wide K slabs per hi*hi register flush (0: library default)
+  int flush;  // K=16 MMAs per hi*hi register flush (0: library default)
   int skip_loads;  // test hook: the producer issues no loads (bounded waits expire)
   GemmOp op[2];
   unsigned* status;  // device status word (non-finite / timeout bits)

@@ -1,28 +1,29 @@
 // Batched split-fp16 GEMM on tcgen05 tensor cores (sm_100a), persistent and
 // warp-specialised.
 //
-// Each CTA (one per SM) walks a static round-robin list of 128 x 128 output
-// tiles of all problems of the launch.  Roles (320 threads):
+// Each CTA (one per SM) walks a static round-robin list of the launch's
+// 128 x 128 output tiles over all problems of the launch.  Roles (448 threads):
 //   warp 0, one lane   TMA producer: streams the A hi/lo and B hi/lo tiles of
 //                      each 64-wide K slab into a 3-stage shared-memory ring
 //                      (A always K-major; B K-major, or MN-major as two
 //                      64-column boxes when the op multiplies by B itself);
 //   warp 1, one lane   MMA issuer;
-//   warps 2-9          epilogue; warp w reads tensor-memory lanes 32*(w%4)..
-//                      and columns 64*((w-2)/4).. of each accumulator, so
-//                      every thread owns 64 columns of one output row.
-// Tensor memory (512 columns): a ring of three 128-column hi*hi accumulators
-// and one 128-column lo accumulator.
+//   warps 2-9          accumulators: warp w reads tensor-memory lanes
+//                      32*(w%4).. and 64 of the 128 columns, so each thread
+//                      sums 64 columns of one output row in registers;
+//   warps 10-13        output: one thread per row writes the finished tile.
 //
-// The tensor core's fp32 accumulation truncates (the bias grows linearly
-// with the number of MMAs accumulated).  The hi*hi products, which carry the
-// result's magnitude, are therefore accumulated in tensor memory over one
-// flush segment only (args.flush K=16 MMAs, default one) and then added
-// with round-to-nearest into fp32 registers of the epilogue warps (packed
-// f32x2 adds), while the MMA warp fills the next ring buffer.  The hi*lo + lo*hi products enter the
-// result scaled by 2^-11 and stay in tensor memory for the whole K range;
-// they are read into the registers as soon as a tile's last MMA retires, so
-// the next tile can start while the epilogue writes the previous one out.
+// The tensor core's fp32 accumulation truncates, so a sum kept in tensor
+// memory over many MMAs drifts low.  Each K=16 step therefore gets a fresh
+// tensor-memory buffer from a ring of three: the MMA warp computes hi*lo +
+// lo*hi into it and then hi*hi with the buffer's content scaled by 2^-11
+// (the MMA's input-scaling operand), so the buffer holds the step's whole
+// product after one truncating addition; the accumulator warps add it into
+// fp32 registers with round-to-nearest (packed f32x2 adds) and release it.
+// At the end of a tile they park the sums in a fourth tensor-memory buffer
+// and go on with the next tile at once, while the output warps apply the
+// epilogue (scales, Cin, identity shift) and store the parked tile: the
+// ring keeps draining while a tile is written out.
 #include "gemm.cuh"
 #include "profile.cuh"
 #include "ptx.cuh"
@@ -35,28 +36,21 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kKBlk = 64;                          // fp16 elements per 128-byte row
-constexpr int kStages = 3;
-constexpr int kTileBytes = kTile * kKBlk * 2;      // 16 KB
+constexpr int kTileBytes = kTile * kKBlk * 2;      // 16 KB per plane and slab
 constexpr int kStageBytes = 4 * kTileBytes;        // A hi, A lo, B hi, B lo
-#ifndef DASH_EPI_WARPS
-#define DASH_EPI_WARPS 8
-#endif
-constexpr int kEpiWarp0 = 2;
-constexpr int kEpiWarps = DASH_EPI_WARPS;          // 4 or 8
-constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr int kCols = kTile * 4 / kEpiWarps;       // accumulator columns per epilogue thread
-constexpr int kRing = 3;                           // hi*hi accumulators
+constexpr int kStages = 3;
+constexpr int kRing = 3;                           // per-K-step product buffers
+constexpr uint32_t kColPark = kRing * 128;         // finished-tile buffer
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColLO = kRing * 128;           // lo accumulator
-#ifndef DASH_FLUSH_MMAS
-#define DASH_FLUSH_MMAS 1
-#endif
-constexpr int kDefaultFlush = DASH_FLUSH_MMAS;     // K=16 MMAs per hi*hi flush
+constexpr int kAccWarp0 = 2, kAccWarps = 8;
+constexpr int kOutWarp0 = kAccWarp0 + kAccWarps, kOutWarps = 4;
+constexpr int kThreads = 32 * (kOutWarp0 + kOutWarps);
+constexpr int kCols = 64;                          // columns summed per accumulator thread
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
-  uint64_t hh_full[kRing], hh_empty[kRing];
-  uint64_t lo_full, lo_empty;
+  uint64_t acc_full[kRing], acc_empty[kRing];
+  uint64_t park_full, park_empty;
   uint64_t drain;
   uint32_t tmem_slot;
   int abort;
@@ -67,17 +61,17 @@ __device__ __forceinline__ int at(const Idx& i, int p) {
   return i.base + (i.stride > 0 ? i.stride : 1) * (i.mod > 0 ? p % i.mod : p);
 }
 
-// Tile t of a problem -> (tile row, tile column).  sym: upper triangle only,
-// enumerated row by row.
-__device__ __forceinline__ void tile_coords(int t, int nt, int sym, int& ti, int& tj) {
+// Tile t of a problem -> (tile row, tile column).  sym: upper triangle of
+// the nt x nt square tile grid only, enumerated row by row.
+__device__ __forceinline__ void tile_coords(int t, int ntn, int sym, int& ti, int& tj) {
   if (!sym) {
-    ti = t / nt;
-    tj = t % nt;
+    ti = t / ntn;
+    tj = t % ntn;
     return;
   }
   int r = 0;
-  while (t >= nt - r) {
-    t -= nt - r;
+  while (t >= ntn - r) {
+    t -= ntn - r;
     ++r;
   }
   ti = r;
@@ -85,13 +79,13 @@ __device__ __forceinline__ void tile_coords(int t, int nt, int sym, int& ti, int
 }
 
 // Flattened tile index -> (op, problem, tile row, tile column).
-__device__ __forceinline__ void decode(const GemmArgs& args, int tpp, int nt, long long t, int& op, int& p,
+__device__ __forceinline__ void decode(const GemmArgs& args, int tpp, int ntn, long long t, int& op, int& p,
                                        int& ti, int& tj) {
   const long long n0 = static_cast<long long>(args.op[0].nprob) * tpp;
   op = t < n0 ? 0 : 1;
   const long long u = op ? t - n0 : t;
   p = static_cast<int>(u / tpp);
-  tile_coords(static_cast<int>(u % tpp), nt, args.sym, ti, tj);
+  tile_coords(static_cast<int>(u % tpp), ntn, args.sym, ti, tj);
 }
 
 __device__ __forceinline__ void fail_timeout(volatile int* abort_flag, unsigned* status) {
@@ -100,8 +94,8 @@ __device__ __forceinline__ void fail_timeout(volatile int* abort_flag, unsigned*
 }
 
 // Descriptor of an MN-major operand tile: 64 K-rows of 128 bytes per
-// 64-column box, two boxes 8 KB apart (leading byte offset), 8-row swizzle
-// atoms of 1024 bytes (stride byte offset), 128-byte swizzle.
+// 64-column box, boxes 8 KB apart (leading byte offset), 8-row swizzle atoms
+// of 1024 bytes (stride byte offset), 128-byte swizzle.
 __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
@@ -176,8 +170,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// FL: K=16 MMAs per hi*hi flush segment (1, 2 or 4), or 0 for one segment per tile.
-template <int FL>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_split_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                       const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -192,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt = args.B / kTile;
   const int tpp = args.sym ? nt * (nt + 1) / 2 : nt * nt;
   const int nk = args.B / kKBlk;
-  const int nseg = FL == 0 ? 1 : nk * (kKBlk / 16) / FL;  // flush segments per tile
+  const int nsteps = nk * (kKBlk / 16);  // K=16 steps per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -200,11 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->empty[s], 1);
     }
     for (int b = 0; b < kRing; ++b) {
-      mbar_init(&bars->hh_full[b], 1);
-      mbar_init(&bars->hh_empty[b], kEpiWarps);
+      mbar_init(&bars->acc_full[b], 1);
+      mbar_init(&bars->acc_empty[b], kAccWarps);
     }
-    mbar_init(&bars->lo_full, 1);
-    mbar_init(&bars->lo_empty, kEpiWarps);
+    mbar_init(&bars->park_full, kAccWarps);
+    mbar_init(&bars->park_empty, kOutWarps);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -244,16 +236,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
           tma_load_3d(st, ta, &bars->full[s], kb * kKBlk, ti * kTile, 2 * am);
           tma_load_3d(st + kTileBytes, ta, &bars->full[s], kb * kKBlk, ti * kTile, 2 * am + 1);
-          if (g.b_mn) {  // rows kb*64.. of B, columns tj*128.. as two 64-column boxes
 #pragma unroll
-            for (int pl = 0; pl < 2; ++pl) {
-              uint8_t* dst = st + (2 + pl) * kTileBytes;
+          for (int pl = 0; pl < 2; ++pl) {
+            uint8_t* dst = st + (2 + pl) * kTileBytes;
+            if (g.b_mn) {  // rows kb*64.. of B, columns tj*128.. as two 64-column boxes
               tma_load_3d(dst, tb, &bars->full[s], tj * kTile, kb * kKBlk, 2 * bm + pl);
               tma_load_3d(dst + kTileBytes / 2, tb, &bars->full[s], tj * kTile + 64, kb * kKBlk, 2 * bm + pl);
+            } else {
+              tma_load_3d(dst, tb, &bars->full[s], kb * kKBlk, tj * kTile, 2 * bm + pl);
             }
-          } else {
-            tma_load_3d(st + 2 * kTileBytes, tb, &bars->full[s], kb * kKBlk, tj * kTile, 2 * bm);
-            tma_load_3d(st + 3 * kTileBytes, tb, &bars->full[s], kb * kKBlk, tj * kTile, 2 * bm + 1);
           }
           if (++s == kStages) {
             s = 0;
@@ -276,51 +267,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t sbase = smem_u32(smem);
       const uint64_t kd0 = sw128_kmajor_desc(sbase), md0 = sw128_mnmajor_desc(sbase);
-      constexpr uint32_t kTileD = kTileBytes >> 4;  // descriptor address units
-      uint32_t s = 0, fpar = 0;                     // stage, parity of its next fill
-      uint32_t hb = 0, hpar = (1u << kRing) - 1u;   // hh buffer, parity bits of the next release per buffer
-      uint32_t lpar = 1u;                           // parity of the lo accumulator's next release
+      constexpr uint32_t kTD = kTileBytes >> 4;   // descriptor address units
+      uint32_t s = 0, fpar = 0;                    // stage, parity of its next fill
+      uint32_t hb = 0, hpar = (1u << kRing) - 1u;  // ring buffer, parity bits of the next release per buffer
       bool ok = true;
-      const uint32_t lo_t = tbase + kColLO;
       for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
         int op, p, ti, tj;
         decode(args, tpp, nt, t, op, p, ti, tj);
         const bool bmn = args.op[op].b_mn != 0;
-        const uint32_t idesc = f16_idesc(128, 128) | (bmn ? (1u << 16) : 0u);
-        const uint64_t bd0 = (bmn ? md0 : kd0) + 2 * kTileD;
+        const uint32_t idesc = f16_idesc(kTile, kTile) | (bmn ? (1u << 16) : 0u);
+        const uint64_t bd0 = (bmn ? md0 : kd0) + 2 * kTD;
         const uint32_t bstep = bmn ? (2048u >> 4) : (32u >> 4);
-        ok = mbar_wait(&bars->lo_empty, lpar, abort_flag);
-        lpar ^= 1u;
-        if (!ok) break;
-        tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
           ok = mbar_wait(&bars->full[s], fpar, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t so = s * (kStageBytes >> 4);
-          const uint64_t ah = kd0 + so, al = ah + kTileD, bh = bd0 + so, bl = bh + kTileD;
+          const uint64_t ah = kd0 + so, al = ah + kTD, bh = bd0 + so, bl = bh + kTD;
 #pragma unroll
           for (int kk = 0; kk < kKBlk / 16; ++kk) {
-            const bool seg_start = FL == 0 ? (kb == 0 && kk == 0) : (kk % FL) == 0;
-            const bool seg_end = FL == 0 ? (kb == nk - 1 && kk == kKBlk / 16 - 1) : (kk % FL) == FL - 1;
-            if (seg_start) {
-              ok = mbar_wait(&bars->hh_empty[hb], (hpar >> hb) & 1u, abort_flag);
-              hpar ^= 1u << hb;
-              if (!ok) break;
-              tc_fence_after();
-            }
+            ok = mbar_wait(&bars->acc_empty[hb], (hpar >> hb) & 1u, abort_flag);
+            hpar ^= 1u << hb;
+            if (!ok) break;
+            tc_fence_after();
             const uint32_t ka = 2u * kk, kbo = bstep * kk;
-            mma_f16_ss(tbase + hb * 128u, ah + ka, bh + kbo, idesc, seg_start ? 0u : 1u);
-            mma_f16_ss(lo_t, ah + ka, bl + kbo, idesc, (kb == 0 && kk == 0) ? 0u : 1u);
-            mma_f16_ss(lo_t, al + ka, bh + kbo, idesc, 1u);
-            if (seg_end) {
-              mma_commit(&bars->hh_full[hb]);
-              hb = hb == kRing - 1 ? 0u : hb + 1u;
-            }
+            const uint32_t d = tbase + hb * 128u;
+            mma_f16_ss(d, ah + ka, bl + kbo, idesc, 0u);         // hi * lo
+            mma_f16_ss(d, al + ka, bh + kbo, idesc, 1u);         // + lo * hi
+            mma_f16_ss_acc_down11(d, ah + ka, bh + kbo, idesc);  // hi * hi + 2^-11 * (...)
+            mma_commit(&bars->acc_full[hb]);
+            hb = hb == kRing - 1 ? 0u : hb + 1u;
           }
           if (!ok) break;
           mma_commit(&bars->empty[s]);
-          if (kb == nk - 1) mma_commit(&bars->lo_full);
           if (++s == kStages) {
             s = 0;
             fpar ^= 1u;
@@ -333,42 +312,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(&bars->drain, 0u, &never);
     }
-  } else {
-    // ---------------------------------------------------------------- epilogue
-    const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
-    const int half = (warp - kEpiWarp0) >> 2;
-    const uint32_t lane_off = (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(half * kCols);
-    const size_t B = static_cast<size_t>(args.B);
-    const size_t BB = B * B;
-    uint32_t hb = 0, hpar = 0, lpar = 0;  // hh buffer and fill parities, lo fill parity
+  } else if (warp < kOutWarp0) {
+    // ---------------------------------------------------------------- accumulators
+    const int quad = warp & 3;                 // tensor-memory lane quadrant of this warp
+    const int cgrp = (warp - kAccWarp0) >> 2;  // 64-column half of the tile
+    const uint32_t lane_off = (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(cgrp * kCols);
+    uint32_t hb = 0, hpar = 0, ppar = 1;  // ring buffer, its fill parities, park release parity
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
-      int op, p, ti, tj;
-      decode(args, tpp, nt, t, op, p, ti, tj);
-      const GemmOp& g = args.op[op];
-      const int row = ti * kTile + quad * 32 + lane;
-      const int cbase = tj * kTile + half * kCols;
-      {  // pull this thread's Cin row segment into L2 while the mainloop runs
-        const size_t prow = static_cast<size_t>(row) * B + static_cast<size_t>(cbase);
-        if (g.cin_split && !g.cin_trans) {
-          const __half* cb = g.cin_split + static_cast<size_t>(at(g.cin_i, p)) * 2 * BB + prow;
-          prefetch_l2(cb);
-          prefetch_l2(cb + BB);
-        }
-        if (g.cin_f32) {
-          const float* cb = g.cin_f32 + static_cast<size_t>(at(g.cinf_i, p)) * BB + prow;
-          prefetch_l2(cb);
-          prefetch_l2(cb + 32);
-        }
-      }
       float S[kCols];
 #pragma unroll
       for (int j = 0; j < kCols; ++j) S[j] = 0.0f;
-
       bool ok = true;
-      for (int sg = 0; sg < nseg; ++sg) {
-        // epilogue warps sleep in the barrier while they wait, leaving the
-        // issue slots of their scheduler to the MMA and TMA threads
-        if (!mbar_wait_sleep(&bars->hh_full[hb], (hpar >> hb) & 1u, abort_flag)) {
+      for (int sg = 0; sg < nsteps; ++sg) {
+        // waiting warps sleep in the barrier, leaving the issue slots of
+        // their scheduler to the MMA and TMA threads
+        if (!mbar_wait_sleep(&bars->acc_full[hb], (hpar >> hb) & 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -376,88 +334,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t src = tbase + lane_off + hb * 128u;
 #pragma unroll
-        for (int c = 0; c < kCols / 64; ++c) {
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(src + 64 * c, r0);
-          tmem_ld_32x32b_x32(src + 64 * c + 32, r1);
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x16(src + 32 * c, r);
+          tmem_ld_32x32b_x16(src + 32 * c + 16, r + 16);
           tmem_ld_wait();
-          if (c + 1 == kCols / 64) {  // registers hold the whole segment now
+          if (c + 1 == kCols / 32) {  // registers hold the whole step now
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->hh_empty[hb]);
+            if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
             hb = hb == kRing - 1 ? 0u : hb + 1u;
           }
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-#ifdef DASH_PLAIN_FADD
-            S[64 * c + j] += __uint_as_float(r0[j]);
-            S[64 * c + j + 1] += __uint_as_float(r0[j + 1]);
-            S[64 * c + 32 + j] += __uint_as_float(r1[j]);
-            S[64 * c + 32 + j + 1] += __uint_as_float(r1[j + 1]);
-#else
-            add_f32x2(S[64 * c + j], S[64 * c + j + 1], r0[j], r0[j + 1]);
-            add_f32x2(S[64 * c + 32 + j], S[64 * c + 32 + j + 1], r1[j], r1[j + 1]);
-#endif
-          }
+          for (int j = 0; j < 32; j += 2) add_f32x2(S[32 * c + j], S[32 * c + j + 1], r[j], r[j + 1]);
         }
       }
+      // hand the tile to the output warps through the park buffer
       if (ok) {
-        ok = mbar_wait_sleep(&bars->lo_full, lpar, abort_flag);
-        lpar ^= 1u;
+        ok = mbar_wait_sleep(&bars->park_empty, ppar, abort_flag);
+        ppar ^= 1u;
       }
       if (!ok) {
-        if (threadIdx.x == kEpiWarp0 * 32) fail_timeout(abort_flag, args.status);
+        if (threadIdx.x == kAccWarp0 * 32) fail_timeout(abort_flag, args.status);
         break;
       }
       tc_fence_after();
-      {
-        const uint32_t src = tbase + lane_off + kColLO;
 #pragma unroll
-        for (int h = 0; h < kCols / 32; ++h) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(src + 32 * h, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) S[32 * h + j] += __uint_as_float(r[j]) * kLoUnscale;
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->lo_empty);  // the next tile may start accumulating
-      }
-
+      for (int c = 0; c < kCols / 16; ++c) tmem_st_32x32b_x16(tbase + lane_off + kColPark + 16 * c, &S[16 * c]);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->park_full);
+    }
+  } else {
+    // ---------------------------------------------------------------- output
+    const int quad = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const size_t B = static_cast<size_t>(args.B);
+    const size_t BB = B * B;
+    uint32_t ppar = 0;
+    for (long long t = blockIdx.x; t < total; t += gridDim.x) {
+      int op, p, ti, tj;
+      decode(args, tpp, nt, t, op, p, ti, tj);
+      const GemmOp& g = args.op[op];
+      const int row = ti * kTile + quad * 32 + lane;
+      const int cbase = tj * kTile;
       const float s = g.scale ? g.scale[at(g.scale_i, p)] : 1.0f;
       const __half* cin = g.cin_split ? g.cin_split + static_cast<size_t>(at(g.cin_i, p)) * 2 * BB : nullptr;
       const float* cinf = g.cin_f32 ? g.cin_f32 + static_cast<size_t>(at(g.cinf_i, p)) * BB : nullptr;
       __half* os = g.out_split ? g.out_split + static_cast<size_t>(at(g.out_i, p)) * 2 * BB : nullptr;
-      __half* ot = g.outt_split ? g.outt_split + static_cast<size_t>(at(g.outt_i, p)) * 2 * BB : nullptr;
       float* of = g.out_f32 ? g.out_f32 + static_cast<size_t>(at(g.outf_i, p)) * BB : nullptr;
-      float* oft = g.outt_f32 ? g.outt_f32 + static_cast<size_t>(at(g.outtf_i, p)) * BB : nullptr;
       const bool mirror = args.sym && (ti != tj);
       BlockDesc bd;
       if (g.blocks) bd = g.blocks[p];
+      SplitChunk nxt;  // Cin is loaded one chunk ahead, the first before the wait
+      if (cin) nxt = ld_chunk(cin, BB, row * B + cbase);
+      if (!mbar_wait_sleep(&bars->park_full, ppar, abort_flag)) {
+        if (threadIdx.x == kOutWarp0 * 32) fail_timeout(abort_flag, args.status);
+        break;
+      }
+      ppar ^= 1u;
+      tc_fence_after();
       bool bad = false;
       float sumsq = 0.0f;
-      const bool cin_rows = cin && !g.cin_trans;
-      SplitChunk nxt;
-      if (cin_rows) nxt = ld_chunk(cin, BB, row * B + cbase);
-
-#pragma unroll
-      for (int c = 0; c < kCols / 16; ++c) {
+#pragma unroll 1
+      for (int c = 0; c < kTile / 16; ++c) {
         const int col0 = cbase + c * 16;
-        float* v = &S[c * 16];  // finished in place
+        float v[16];
+        tmem_ld_32x32b_x16(tbase + lane_off + kColPark + 16 * c, reinterpret_cast<uint32_t*>(v));
+        tmem_ld_wait();
+        if (c + 1 == kTile / 16) {  // the park buffer is free for the next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->park_empty);
+        }
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] *= g.alpha;
-        if (cin_rows) {  // this chunk's Cin was loaded one chunk ahead
+        if (cin) {
           const SplitChunk cur = nxt;
-          if (c + 1 < kCols / 16) nxt = ld_chunk(cin, BB, row * B + col0 + 16);
+          if (c + 1 < kTile / 16) nxt = ld_chunk(cin, BB, row * B + col0 + 16);
           float cj[16];
           join_chunk(cur, cj);
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] += g.beta * cj[j];
-        } else if (cin) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[j] += g.beta * join_f16(cin[(col0 + j) * B + row], cin[BB + (col0 + j) * B + row]);
         }
         if (cinf) {
           const float4* c4 = reinterpret_cast<const float4*>(cinf + row * B + col0);
@@ -497,7 +456,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_split16(os, BB, row * B + col0, v, bad);
           if (mirror) store_split16_t(os, B, BB, row, col0, v, bad);
         }
-        if (ot) store_split16_t(ot, B, BB, row, col0, v, bad);
         if (of) {
           float4* d4 = reinterpret_cast<float4*>(of + row * B + col0);
 #pragma unroll
@@ -506,10 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) of[(col0 + j) * B + row] = v[j];
           }
-        }
-        if (oft) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) oft[(col0 + j) * B + row] = v[j];
         }
       }
       if (bad) atomicOr(args.status, kStatusNonFinite);
@@ -550,22 +504,15 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   if (g_load_fault.exchange(0) != 0) a.skip_loads = 1;
   CUtensorMap maps[4];
   for (int o = 0; o < 2; ++o) {
-    const OpBuffers& b = bufs[o < args.nops ? o : 0];
-    cudaError_t e = encode_split_stack_map(&maps[2 * o], b.a, a.B, b.a_nmat, 128);
+    const OpBuffers& b = bufs[o < a.nops ? o : 0];
+    cudaError_t e = encode_split_stack_map(&maps[2 * o], b.a, a.B, b.a_nmat, kTile);
     if (e != cudaSuccess) return e;
-    e = encode_split_stack_map(&maps[2 * o + 1], b.b, a.B, b.b_nmat, a.op[o].b_mn ? 64 : 128);
+    e = encode_split_stack_map(&maps[2 * o + 1], b.b, a.B, b.b_nmat, a.op[o].b_mn ? 64 : kTile);
     if (e != cudaSuccess) return e;
   }
-  const int nm = (a.B / kKBlk) * (kKBlk / 16);  // K=16 MMAs per tile
-  if (a.flush <= 0) a.flush = kDefaultFlush;
-  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmArgs,
-               const long long) = a.flush >= nm  ? gemm_split_kernel<0>
-                                  : a.flush >= 4 ? gemm_split_kernel<4>
-                                  : a.flush >= 2 ? gemm_split_kernel<2>
-                                                 : gemm_split_kernel<1>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(gemm_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int nt = a.B / kTile;
+  const long long nt = a.B / kTile;
   const long long tpp = a.sym ? nt * (nt + 1) / 2 : nt * nt;
   const long long total = tpp * nprob;
   const long long sms = sm_count();
@@ -573,7 +520,7 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   // useful flops: each computed 128 x 128 tile is one 2*128*128*B product
   const double flops = 2.0 * kTile * kTile * static_cast<double>(a.B) * static_cast<double>(total);
   const int slot = prof_begin(kProfGemm, stream, flops);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
+  gemm_split_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

@@ -3,10 +3,10 @@
 // Every product on the hot path of the batched block-Shampoo step is a
 // B x B x B product of two matrices from stacked (N, B, B) tensors (the DASH
 // explainer's "Building blocks": stack blocks into (N, B, B), run batched
-// products).  Operands are held as two fp16 planes (hi, lo * 2^11) and the
-// kernel accumulates hi*hi and hi*lo + lo*hi in two fp32 tensor-memory
-// accumulators (tcgen05, kind::f16), which gives about fp32 accuracy at the
-// fp16 tensor-core rate.
+// products).  Operands are held as two fp16 planes (hi, lo * 2^11); for every
+// K=16 step the kernel computes hi*lo + lo*hi and then hi*hi + 2^-11 * that in
+// fp32 tensor memory (tcgen05, kind::f16) and adds the step's product into
+// fp32 registers, which gives about fp32 accuracy at the fp16 tensor-core rate.
 //
 // Problem p computes
 //     out_p = s_p * (alpha * A_p op(B_p) + beta * Cin_p + gamma * I)
@@ -50,17 +50,12 @@ struct GemmOp {
   Idx scale_i;
   const __half* cin_split;   // split Cin stack (nullptr: none)
   Idx cin_i;
-  int cin_trans;             // 1: Cin_p(r, c) is read from element (c, r)
   const float* cin_f32;      // fp32 Cin stack (nullptr: none)
   Idx cinf_i;
-  __half* out_split;         // split output, as computed (+ mirror if sym)
+  __half* out_split;         // split output (+ mirror if sym)
   Idx out_i;
-  __half* outt_split;        // split output, transposed (non-sym only)
-  Idx outt_i;
-  float* out_f32;            // fp32 output, as computed (+ mirror if sym)
+  float* out_f32;            // fp32 output (+ mirror if sym)
   Idx outf_i;
-  float* outt_f32;           // fp32 output, transposed (non-sym only)
-  Idx outtf_i;
   const BlockDesc* blocks;   // non-null: scatter out_p into u_out (parameter layout)
   float* u_out;
   float* unorm;              // per-problem sum of squares of the scattered out_p
@@ -70,7 +65,6 @@ struct GemmArgs {
   int B;      // matrix size; multiple of 128
   int sym;    // 1: symmetric outputs (upper-triangle tiles + mirrored writes)
   int nops;   // 1 or 2
-  int flush;  // K=16 MMAs per hi*hi register flush (0: library default)
   int skip_loads;  // test hook: the producer issues no loads (bounded waits expire)
   GemmOp op[2];
   unsigned* status;  // device status word (non-finite / timeout bits)

@@ -78,9 +78,19 @@ __device__ __forceinline__ void tile_coords(int t, int ntn, int sym, int& ti, in
   tj = r + t;
 }
 
-// Flattened tile index -> (op, problem, tile row, tile column).
+// Flattened tile index -> (op, problem, tile row, tile column).  When both
+// ops of a launch have the same problems, the two ops of a problem are
+// adjacent in the order, so operands they share are read from L2 once.
 __device__ __forceinline__ void decode(const GemmArgs& args, int tpp, int ntn, long long t, int& op, int& p,
                                        int& ti, int& tj) {
+  if (args.op[1].nprob == args.op[0].nprob) {
+    const long long pair = 2ll * tpp;
+    p = static_cast<int>(t / pair);
+    const int r = static_cast<int>(t - static_cast<long long>(p) * pair);
+    op = r >= tpp ? 1 : 0;
+    tile_coords(op ? r - tpp : r, ntn, args.sym, ti, tj);
+    return;
+  }
   const long long n0 = static_cast<long long>(args.op[0].nprob) * tpp;
   op = t < n0 ? 0 : 1;
   const long long u = op ? t - n0 : t;

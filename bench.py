@@ -54,6 +54,9 @@ def parse_args():
     p.add_argument("--iters", type=int, default=None, help="Newton-DB iterations per stage")
     p.add_argument("--degree", type=int, default=16)
     p.add_argument("--n", type=int, default=256, help="matrices in the standalone-roots workload")
+    p.add_argument("--root-every", type=int, default=1,
+                   help="recompute roots every F-th step and reuse them in between (default: every step)")
+    p.add_argument("--scaling", default="spectral", choices=["spectral", "frobenius"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -302,7 +305,8 @@ def main():
         grads = make_grads(spec, dev, seed=0)
         params = [torch.randn(g.shape, device=dev) * 0.02 for g in grads]
         hp = bd.make_hparams(block_size=B, solver=solver, ndb_iters1=iters, ndb_iters2=iters,
-                             cheb_degree=args.degree)
+                             cheb_degree=args.degree, root_every=args.root_every,
+                             scaling=bd.SCALING_FROBENIUS if args.scaling == "frobenius" else bd.SCALING_SPECTRAL)
         opt = bd.Shampoo(params, grads, hp=hp,
                          v0=torch.from_numpy(wl.pi_start_vectors(B, 32, seed=0)).to(dev))
         bsz = block_sizes(spec["shapes"], B)
@@ -423,14 +427,19 @@ def main():
     padded = 2.0 * B ** 3 * gemms * n_factors
     unpadded = sum(2.0 * b ** 3 * gemms for b in factor_sizes)
     tf32_peak = tensor_peak / 2.0
-    root_s = s_ms * 1e-3 / args.steps
-    inverse_root = {"ms_per_step": round(root_s * 1e3, 3),
-                    "tflops": round(padded / root_s / 1e12, 1),
-                    "tflops_unpadded": round(unpadded / root_s / 1e12, 1),
-                    "tf32_peak_tflops": tf32_peak,
-                    "frac_of_tf32_peak": round(padded / root_s / 1e12 / tf32_peak, 4),
-                    "frac_of_tf32_peak_unpadded": round(unpadded / root_s / 1e12 / tf32_peak, 4),
-                    "peak_kind": f"{peak_kind}: bf16 sustained x 0.5 (nominal TF32/BF16 ratio)"}
+    # timed steps are W+1 .. W+K; roots are computed on steps with (t-1) % f == 0
+    every = max(1, args.root_every) if spec["shapes"] is not None else 1
+    root_steps = sum(1 for t in range(args.warmup + 1, args.warmup + args.steps + 1) if (t - 1) % every == 0)
+    inverse_root = None
+    if root_steps and s_ms > 0:
+        root_s = s_ms * 1e-3 / root_steps
+        inverse_root = {"ms_per_root_step": round(root_s * 1e3, 3), "root_steps_timed": root_steps,
+                        "tflops": round(padded / root_s / 1e12, 1),
+                        "tflops_unpadded": round(unpadded / root_s / 1e12, 1),
+                        "tf32_peak_tflops": tf32_peak,
+                        "frac_of_tf32_peak": round(padded / root_s / 1e12 / tf32_peak, 4),
+                        "frac_of_tf32_peak_unpadded": round(unpadded / root_s / 1e12 / tf32_peak, 4),
+                        "peak_kind": f"{peak_kind}: bf16 sustained x 0.5 (nominal TF32/BF16 ratio)"}
     stages = {k: round(v[0] / args.steps, 3) for k, v in prof.items() if isinstance(v, tuple) and k != "gemm"}
 
     cpu = None
@@ -445,7 +454,9 @@ def main():
             "config": dict({"workload": spec["desc"], "block_size": B, "solver": args.solver,
                             "iters_per_stage": iters if args.solver == "ndb" else None,
                             "cheb_degree": args.degree if args.solver == "cheb" else None,
-                            "power_iteration": "10 products x 32 starts",
+                            "scale_estimate": ("power iteration, 10 products x 32 starts" if args.scaling == "spectral"
+                                               else "Frobenius norm"),
+                            "roots_every_steps": max(1, args.root_every),
                             "l2": "working set far larger than the 126 MB L2 (no flush needed)",
                             "parallelism": f"replicas x{world}"}, **ctx_info),
             "roofline": roofline, "inverse_root": inverse_root, "stage_ms": stages,

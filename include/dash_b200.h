@@ -61,6 +61,12 @@ extern "C" {
 #define SHAMPOO_SOLVER_NEWTON_DB 0
 #define SHAMPOO_SOLVER_CHEBYSHEV 1
 
+/* Scale estimate lambda each factor is divided by (c = 1 / (2 lambda)) before
+ * the root solver ("Building blocks", scaling): the multi-start power
+ * iteration's spectral estimate, or the Frobenius norm ||F + eps I||_F. */
+#define SHAMPOO_SCALING_SPECTRAL 0
+#define SHAMPOO_SCALING_FROBENIUS 1
+
 /* Bits of the workspace status word. */
 #define SHAMPOO_STATUS_NONFINITE 1u
 #define SHAMPOO_STATUS_TIMEOUT 2u
@@ -93,6 +99,9 @@ typedef struct {
   float cheb_delta; /* Chebyshev interval [delta, 1 + delta] */
   int pi_starts;    /* power-iteration start vectors K; must be 32 */
   int pi_iters;     /* power-iteration products, 1..100 */
+  int root_every;   /* roots recomputed every root_every-th step (steps 1, 1 + f, ...);
+                       other steps reuse the roots kept in the workspace (0 or 1: every step) */
+  int scaling;      /* SHAMPOO_SCALING_* */
 } shampoo_hparams;
 
 /* Build the block table for a parameter set (host only; no device work).
@@ -136,6 +145,11 @@ SHAMPOO_API int shampoo_accumulate(shampoo_ctx* ctx, float* factors, void* ws, s
  *   m, v (bias-corrected with `step` >= 1); P = m_hat / (sqrt(v_hat) + adam_eps);
  *   s = ||P_b||_F / ||U_b||_F (0 when U_b = 0); param -= lr * s * U_b.
  * Requires shampoo_accumulate on the same ws earlier in the same step.
+ * Roots are computed on root steps, (step - 1) % root_every == 0, and on any
+ * step whose ws does not hold this ctx's roots yet; other steps precondition
+ * with the roots kept in ws since the last root step (the factors, moments
+ * and parameters are still updated every step), and leave lambda_out and
+ * roots_out untouched.
  * `lambda_out` (device, n_factors floats, or NULL) receives the estimates.
  * `roots_out` (device, (n_factors, B, B) fp32, or NULL) receives X. */
 SHAMPOO_API int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const float* v0, int step,
@@ -149,6 +163,8 @@ SHAMPOO_API int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors
  *   stage 1: Y = c A_i', Z = I, iters1 times E = (3I - ZY)/2, Y <- YE, Z <- EZ;
  *   stage 2: the same from Y = Y(stage 1), Z = I, iters2 times;
  *   X_i = c^(1/4) Z  ~  (A_i + eps I)^(-1/4).
+ * pi_iters = 0 selects Frobenius scaling instead: lambda_i = ||A_i'||_F (v0 is
+ * then not read but must still be a valid pointer).
  * A (device, (n, B, B) fp32, symmetric, read only), X (device, (n, B, B) fp32,
  * written), lambda_out (device, n floats, or NULL).
  * Errors: SHAMPOO_EINVAL, SHAMPOO_EUNSUPPORTED, SHAMPOO_EWORKSPACE, SHAMPOO_ECUDA. */

@@ -22,6 +22,8 @@ SHAMPOO_ENONFINITE = -5
 SHAMPOO_ETIMEOUT = -6
 SOLVER_NEWTON_DB = 0
 SOLVER_CHEBYSHEV = 1
+SCALING_SPECTRAL = 0
+SCALING_FROBENIUS = 1
 PI_STARTS = 32
 
 
@@ -41,14 +43,17 @@ class ShampooHParams(ctypes.Structure):
                 ("init_scale", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("adam_eps", ctypes.c_float), ("lr", ctypes.c_float), ("solver", ctypes.c_int),
                 ("ndb_iters1", ctypes.c_int), ("ndb_iters2", ctypes.c_int), ("cheb_degree", ctypes.c_int),
-                ("cheb_delta", ctypes.c_float), ("pi_starts", ctypes.c_int), ("pi_iters", ctypes.c_int)]
+                ("cheb_delta", ctypes.c_float), ("pi_starts", ctypes.c_int), ("pi_iters", ctypes.c_int),
+                ("root_every", ctypes.c_int), ("scaling", ctypes.c_int)]
 
 
 def make_hparams(block_size=1024, beta=0.95, eps=1e-6, init_scale=1e-6, beta1=0.9, beta2=0.999,
                  adam_eps=1e-8, lr=1e-3, solver=SOLVER_NEWTON_DB, ndb_iters1=14, ndb_iters2=14,
-                 cheb_degree=16, cheb_delta=1e-3, pi_starts=PI_STARTS, pi_iters=10):
+                 cheb_degree=16, cheb_delta=1e-3, pi_starts=PI_STARTS, pi_iters=10, root_every=1,
+                 scaling=SCALING_SPECTRAL):
     return ShampooHParams(block_size, beta, eps, init_scale, beta1, beta2, adam_eps, lr, solver,
-                          ndb_iters1, ndb_iters2, cheb_degree, cheb_delta, pi_starts, pi_iters)
+                          ndb_iters1, ndb_iters2, cheb_degree, cheb_delta, pi_starts, pi_iters, root_every,
+                          scaling)
 
 
 _lib = None

@@ -302,16 +302,20 @@ int run_roots(const float* F, int nf, int B, float eps, const int* fsize, const 
   float* W[2] = {reinterpret_cast<float*>(ws + L.w0), reinterpret_cast<float*>(ws + L.w1)};
   const size_t sstride = static_cast<size_t>(nf) * 3 * dash::kPiStarts;
 
-  // ---- multi-start power iteration ("Building blocks", Multi-Power-Iteration)
   const int pslot = dash::prof_begin(dash::kProfPowerIter, st);
-  DASH_TRY(cudaMemsetAsync(stats, 0, sizeof(float) * sstride * pi_iters, st));
-  for (int t = 0; t < pi_iters; ++t) {
-    dash::launch_pi_iter(F, nf, B, eps, fsize, v0, t ? W[(t - 1) & 1] : nullptr,
-                         t ? stats + (t - 1) * sstride : nullptr, W[t & 1], stats + t * sstride, st);
+  if (pi_iters == 0) {  // Frobenius scaling: lambda = ||F + eps I||_F
+    dash::launch_frob_norm(F, nf, B, eps, fsize, lam, lam_out, st);
+    DASH_LAUNCHED();
+  } else {  // multi-start power iteration ("Building blocks", Multi-Power-Iteration)
+    DASH_TRY(cudaMemsetAsync(stats, 0, sizeof(float) * sstride * pi_iters, st));
+    for (int t = 0; t < pi_iters; ++t) {
+      dash::launch_pi_iter(F, nf, B, eps, fsize, v0, t ? W[(t - 1) & 1] : nullptr,
+                           t ? stats + (t - 1) * sstride : nullptr, W[t & 1], stats + t * sstride, st);
+      DASH_LAUNCHED();
+    }
+    dash::launch_pi_finalize(stats + (pi_iters - 1) * sstride, nf, lam, lam_out, st);
     DASH_LAUNCHED();
   }
-  dash::launch_pi_finalize(stats + (pi_iters - 1) * sstride, nf, lam, lam_out, st);
-  DASH_LAUNCHED();
   dash::prof_end(pslot, st);
 
   const int sslot = dash::prof_begin(dash::kProfSolver, st);
@@ -363,6 +367,7 @@ struct shampoo_ctx {
   size_t off_gs = 0, off_roots = 0, off_u = 0, off_pn = 0, off_un = 0, off_blocks = 0, off_params = 0,
          off_prefix = 0, off_fsize = 0, total = 0;
   const void* tables_ws = nullptr;
+  const void* roots_ws = nullptr;  // workspace holding the roots of the last root step
 };
 
 namespace {
@@ -395,6 +400,8 @@ int check_hparams(const shampoo_hparams* hp) {
   if (hp->cheb_degree < 2 || hp->cheb_degree > 256 || !(hp->cheb_delta > 0.0f) || !std::isfinite(hp->cheb_delta))
     return SHAMPOO_EINVAL;
   if (hp->pi_starts != dash::kPiStarts || hp->pi_iters < 1 || hp->pi_iters > 100) return SHAMPOO_EINVAL;
+  if (hp->root_every < 0 || (hp->scaling != SHAMPOO_SCALING_SPECTRAL && hp->scaling != SHAMPOO_SCALING_FROBENIUS))
+    return SHAMPOO_EINVAL;
   return SHAMPOO_OK;
 }
 
@@ -558,9 +565,14 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   unsigned* status = reinterpret_cast<unsigned*>(ws + ctx->roots.status);
   const int* fsize = reinterpret_cast<const int*>(ws + ctx->off_fsize);
   __half* roots = split_at(ws, ctx->off_roots, 0, B);
-  rc = run_roots(factors, nf, B, hp.eps, fsize, v0, hp.pi_iters, hp.solver, hp.ndb_iters1, hp.ndb_iters2,
-                 hp.cheb_degree, hp.cheb_delta, lambda_out, roots_out, roots, ws, ctx->roots, status, st);
-  if (rc) return rc;
+  const int every = hp.root_every > 0 ? hp.root_every : 1;
+  if ((step - 1) % every == 0 || ctx->roots_ws != ws_v) {  // root step (or no roots kept in this ws yet)
+    const int pi = hp.scaling == SHAMPOO_SCALING_FROBENIUS ? 0 : hp.pi_iters;
+    rc = run_roots(factors, nf, B, hp.eps, fsize, v0, pi, hp.solver, hp.ndb_iters1, hp.ndb_iters2, hp.cheb_degree,
+                   hp.cheb_delta, lambda_out, roots_out, roots, ws, ctx->roots, status, st);
+    if (rc) return rc;
+    ctx->roots_ws = ws_v;
+  }
 
   float* pn = reinterpret_cast<float*>(ws + ctx->off_pn);
   float* un = reinterpret_cast<float*>(ws + ctx->off_un);
@@ -627,7 +639,7 @@ static int inv_root_common(const float* A, float* X, int n, int B, float eps, co
   if (!A || !X || !v0) return SHAMPOO_EINVAL;
   if (n < 1 || !valid_B(B)) return SHAMPOO_EUNSUPPORTED;
   if (n > 32767) return SHAMPOO_EUNSUPPORTED;
-  if (!finite_nonneg(eps) || pi_iters < 1 || pi_iters > 100) return SHAMPOO_EINVAL;
+  if (!finite_nonneg(eps) || pi_iters < 0 || pi_iters > 100) return SHAMPOO_EINVAL;
   const int rc = check_ws(ws, ws_bytes, shampoo_inv_root_workspace_bytes(n, B, solver));
   if (rc) return rc;
   Bump b;

@@ -176,10 +176,6 @@ __device__ __forceinline__ void join_chunk(const SplitChunk& c, float* out) {
   }
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_split_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                       const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,

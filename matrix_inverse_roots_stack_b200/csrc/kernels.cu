@@ -179,6 +179,41 @@ __global__ void pi_finalize_kernel(const float* __restrict__ s, int nf, float* _
   if (lam_out) lam_out[f] = best;
 }
 
+// Frobenius-norm scale estimate ("Building blocks", scaling: the Frobenius
+// alternative to spectral scaling): lambda_f = ||F_f + eps I||_F over the
+// factor's real b x b part (padding excluded).  One CTA per factor, float64
+// accumulation; sum of squares of F plus 2 eps tr(F) + b eps^2.
+__global__ void frob_norm_kernel(const float* __restrict__ F, int B, float eps, const int* __restrict__ fsize,
+                                 float* __restrict__ lam, float* __restrict__ lam_out) {
+  const int f = blockIdx.x;
+  const int b = fsize ? fsize[f] : B;
+  const float* A = F + static_cast<size_t>(f) * B * B;
+  double ss = 0.0, tr = 0.0;
+  for (int i = threadIdx.y; i < b; i += blockDim.y) {
+    const float* row = A + static_cast<size_t>(i) * B;
+    for (int j = threadIdx.x; j < b; j += blockDim.x) {
+      const double x = row[j];
+      ss += x * x;
+      if (j == i) tr += x;
+    }
+  }
+  ss += 2.0 * static_cast<double>(eps) * tr;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  __shared__ double part[32];
+  const int w = (threadIdx.y * blockDim.x + threadIdx.x) >> 5, nw = (blockDim.x * blockDim.y) >> 5;
+  if ((threadIdx.x & 31) == 0) part[w] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0 && threadIdx.y == 0) {
+    double t = 0.0;
+    for (int k = 0; k < nw; ++k) t += part[k];
+    t += static_cast<double>(b) * static_cast<double>(eps) * static_cast<double>(eps);
+    const float v = static_cast<float>(sqrt(t > 0.0 ? t : 0.0));
+    lam[f] = v;
+    if (lam_out) lam_out[f] = v;
+  }
+}
+
 // ------------------------------------------------------------ solver prologues
 
 __device__ __forceinline__ void store_split4(__half* base, size_t BB, size_t idx, const float* x) {
@@ -455,6 +490,12 @@ void launch_pi_iter(const float* F, int nf, int B, float eps, const int* fsize, 
 
 void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* lambda_out, cudaStream_t st) {
   pi_finalize_kernel<<<(nf + 127) / 128, 128, 0, st>>>(stats_last, nf, lambda, lambda_out);
+  prof_count_launch();
+}
+
+void launch_frob_norm(const float* F, int nf, int B, float eps, const int* fsize, float* lambda, float* lambda_out,
+                      cudaStream_t st) {
+  frob_norm_kernel<<<nf, dim3(128, 8), 0, st>>>(F, B, eps, fsize, lambda, lambda_out);
   prof_count_launch();
 }
 

@@ -38,6 +38,11 @@ void launch_pi_iter(const float* F, int nf, int B, float eps, const int* fsize, 
 // lambda[f] = max_j (V.W)_j / (V.V)_j from the last product's statistics.
 void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* lambda_out, cudaStream_t st);
 
+// lambda_f = ||F_f + eps I||_F over the real fsize[f] x fsize[f] part (the
+// Frobenius scale estimate, in place of the power iteration).
+void launch_frob_norm(const float* F, int nf, int B, float eps, const int* fsize, float* lambda, float* lambda_out,
+                      cudaStream_t st);
+
 // Newton-DB stage-1 prologue: c = 1/(2 lambda); Y0 = c (F + eps I) (padding:
 // identity); D0 = (I - Y0)/2; Zhat1 = (I + D0)/zs; xscale = c^(1/4) zs.
 void launch_ndb_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, float zs,

@@ -28,6 +28,13 @@ class HParams:
     adam_eps=1e-8), per-block grafting, power iteration with ``pi_iters``
     products, Newton-DB ``ndb_iters1`` + ``ndb_iters2`` iterations, Chebyshev
     degree ``cheb_degree`` on [cheb_delta, 1 + cheb_delta].
+
+    ``scaling``: the scale estimate of each factor ("Building blocks",
+    scaling): "spectral" (multi-start power iteration) or "frobenius"
+    (lambda = ||L + eps I||_F, which bounds lambda_max from above).
+    ``root_every``: roots are recomputed on steps 1, 1 + f, 1 + 2f, ... and
+    reused in between, while the factors, moments and parameters are updated
+    every step (the update-frequency variant the pages time).
     """
     block_size: int = 128
     beta: float = 0.95
@@ -44,6 +51,8 @@ class HParams:
     cheb_delta: float = 1e-3
     pi_iters: int = 10
     root_level: int = 2          # 1 exact, 2 truncated method (spectral), 3 matmul
+    scaling: str = "spectral"    # "spectral" | "frobenius"
+    root_every: int = 1
 
 
 def block_grid(rows, cols, B):
@@ -81,7 +90,12 @@ def inverse_fourth_root(Abar, V0, hp, lam_est=None):
     """
     b = Abar.shape[0]
     if lam_est is None:
-        lam_est, _ = roots.power_iteration(Abar, V0[:b], hp.pi_iters)
+        if hp.scaling == "frobenius":
+            lam_est = float(np.linalg.norm(Abar, "fro"))
+        elif hp.scaling == "spectral":
+            lam_est, _ = roots.power_iteration(Abar, V0[:b], hp.pi_iters)
+        else:
+            raise ValueError("unknown scaling")
     if hp.solver == "ndb":
         if hp.root_level == 1:
             X = roots.inv_root_eigh(Abar, 4)
@@ -150,9 +164,12 @@ def shampoo_step(thetas, grads, state, hp, V0, lam_override=None):
     order: factor 2k is its L, 2k+1 its R).
 
     Returns (new_thetas, new_state, info) with info = {"lam": [...],
-    "graft": [...], "U": [...], "P": [...]}.
+    "graft": [...], "U": [...], "P": [...], "root_step": bool}; on steps that
+    reuse roots, "lam" holds the estimates of the step that computed them.
     """
     t = state["t"] + 1
+    f_every = max(1, int(hp.root_every))
+    root_step = (t - 1) % f_every == 0
     new_thetas, new_params = [], []
     lam_out, graft_out, U_out, P_out = [], [], [], []
     f = 0
@@ -165,13 +182,16 @@ def shampoo_step(thetas, grads, state, hp, V0, lam_override=None):
         for (r0, r1, c0, c1), blk in zip(block_grid(*th.shape, hp.block_size), ps["blocks"]):
             Gb = G[r0:r1, c0:c1]
             L, R = factor_ema(blk["L"], blk["R"], Gb, hp.beta)
-            new_blocks.append({"L": L, "R": R})
-            XL, lamL = inverse_fourth_root(
-                L + hp.eps * np.eye(L.shape[0]), V0, hp,
-                None if lam_override is None else lam_override[f])
-            XR, lamR = inverse_fourth_root(
-                R + hp.eps * np.eye(R.shape[0]), V0, hp,
-                None if lam_override is None else lam_override[f + 1])
+            if root_step or "XL" not in blk:
+                XL, lamL = inverse_fourth_root(
+                    L + hp.eps * np.eye(L.shape[0]), V0, hp,
+                    None if lam_override is None else lam_override[f])
+                XR, lamR = inverse_fourth_root(
+                    R + hp.eps * np.eye(R.shape[0]), V0, hp,
+                    None if lam_override is None else lam_override[f + 1])
+            else:  # reuse the roots of the last root step
+                XL, XR, lamL, lamR = blk["XL"], blk["XR"], blk["lamL"], blk["lamR"]
+            new_blocks.append({"L": L, "R": R, "XL": XL, "XR": XR, "lamL": lamL, "lamR": lamR})
             lam_out += [lamL, lamR]
             f += 2
             Ub = XL @ Gb @ XR
@@ -183,7 +203,7 @@ def shampoo_step(thetas, grads, state, hp, V0, lam_override=None):
         new_params.append({"blocks": new_blocks, "m": m, "v": v})
         U_out.append(U_full)
         P_out.append(P)
-    info = {"lam": lam_out, "graft": graft_out, "U": U_out, "P": P_out}
+    info = {"lam": lam_out, "graft": graft_out, "U": U_out, "P": P_out, "root_step": root_step}
     return new_thetas, {"params": new_params, "t": t}, info
 
 

@@ -106,6 +106,9 @@ def test_init_blocks_rejects_bad_arguments(lib):
     assert init(lib, [(4, 4)], ndb_iters1=0)[0] == bd.SHAMPOO_EINVAL
     assert init(lib, [(4, 4)], cheb_degree=1)[0] == bd.SHAMPOO_EINVAL
     assert init(lib, [(4, 4)], solver=7)[0] == bd.SHAMPOO_EINVAL
+    assert init(lib, [(4, 4)], root_every=-1)[0] == bd.SHAMPOO_EINVAL
+    assert init(lib, [(4, 4)], scaling=2)[0] == bd.SHAMPOO_EINVAL
+    assert init(lib, [(4, 4)], root_every=5, scaling=bd.SCALING_FROBENIUS)[0] == bd.SHAMPOO_OK
     assert init(lib, [(0, 4)])[0] == bd.SHAMPOO_EINVAL
     ctx = ctypes.c_void_p()
     n = ctypes.c_size_t()
@@ -131,7 +134,8 @@ def test_root_calls_validate_before_device_work(lib):
     assert ndb(p, p, 0, 256, 8, 8, 0.0, p, 10, None, ws, need, None) == bd.SHAMPOO_EUNSUPPORTED
     assert ndb(p, p, 4, 256, 0, 8, 0.0, p, 10, None, ws, need, None) == bd.SHAMPOO_EINVAL
     assert ndb(p, p, 4, 256, 8, 8, -1.0, p, 10, None, ws, need, None) == bd.SHAMPOO_EINVAL
-    assert ndb(p, p, 4, 256, 8, 8, 0.0, p, 0, None, ws, need, None) == bd.SHAMPOO_EINVAL
+    assert ndb(p, p, 4, 256, 8, 8, 0.0, p, -1, None, ws, need, None) == bd.SHAMPOO_EINVAL
+    assert ndb(p, p, 4, 256, 8, 8, 0.0, p, 101, None, ws, need, None) == bd.SHAMPOO_EINVAL
     assert ndb(p, p, 4, 256, 8, 8, 0.0, p, 10, None, None, need, None) == bd.SHAMPOO_EWORKSPACE
     assert ndb(p, p, 4, 256, 8, 8, 0.0, p, 10, None, ws, need - 1, None) == bd.SHAMPOO_EWORKSPACE
     assert ndb(p, p, 4, 256, 8, 8, 0.0, p, 10, None, ctypes.c_void_p(0x100010), need,

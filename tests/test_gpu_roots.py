@@ -152,3 +152,15 @@ def test_bounded_wait_reports_timeout_and_context_survives(torch):
     assert rc == 0
     ref = roots.ndb_inv4root_spectral(A[0].astype(np.float64), lam[0], 6, 6)
     assert rel(X[0], ref) < ROOT_TOL
+
+
+def test_frobenius_scaling_roots(torch):
+    # pi_iters = 0: lambda = ||A + eps I||_F instead of the power iteration
+    A = workloads.spd_stack_geometric(3, 256, 1e3, seed=13)
+    X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=20, iters2=16, eps=1e-6, pi_iters=0)
+    assert rc == 0
+    for i in range(3):
+        ref = np.linalg.norm(A[i].astype(np.float64) + 1e-6 * np.eye(256), "fro")
+        assert abs(lam[i] - ref) <= 1e-5 * ref, (i, lam[i], ref)
+    for i, r in enumerate(ndb_level2(A, 1e-6, lam, 20, 16)):
+        assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))

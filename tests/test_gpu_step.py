@@ -31,7 +31,8 @@ def run_gpu(torch, thetas, grads, hp, steps=1, seed=0):
                         beta1=hp.beta1, beta2=hp.beta2, adam_eps=hp.adam_eps, lr=hp.lr,
                         solver=bd.SOLVER_NEWTON_DB if hp.solver == "ndb" else bd.SOLVER_CHEBYSHEV,
                         ndb_iters1=hp.ndb_iters1, ndb_iters2=hp.ndb_iters2, cheb_degree=hp.cheb_degree,
-                        cheb_delta=hp.cheb_delta, pi_iters=hp.pi_iters)
+                        cheb_delta=hp.cheb_delta, pi_iters=hp.pi_iters, root_every=hp.root_every,
+                        scaling=bd.SCALING_FROBENIUS if hp.scaling == "frobenius" else bd.SCALING_SPECTRAL)
     P = [torch.from_numpy(np.ascontiguousarray(t, dtype=np.float32)).cuda() for t in thetas]
     G = [torch.from_numpy(np.ascontiguousarray(g[0], dtype=np.float32)).cuda() for g in grads]
     v0 = torch.from_numpy(workloads.pi_start_vectors(hp.block_size, 32, seed=seed)).cuda()
@@ -154,3 +155,38 @@ def test_two_steps_block_256(torch):
     hp = ostep.HParams(block_size=256, ndb_iters1=14, ndb_iters2=14, eps=1e-5)
     gpu = run_gpu(torch, th, grads, hp, steps=2)
     compare(gpu, th, grads, hp, steps=2)
+
+
+def test_root_every_reuses_roots(torch):
+    # roots on steps 1 and 3 only (root_every = 2): step 2 and 4 precondition
+    # with the roots kept in the workspace, while factors, moments and
+    # parameters move every step; the oracle caches its roots the same way
+    shapes = [(300, 200), (128, 256)]
+    gs = [workloads.gaussian_gradients(shapes, std=0.1, seed=20 + s) for s in range(4)]
+    grads = [[gs[s][i] for s in range(4)] for i in range(len(shapes))]
+    th = workloads.parameters(shapes, seed=21)
+    hp = ostep.HParams(block_size=128, ndb_iters1=14, ndb_iters2=14, eps=1e-4, root_every=2)
+    gpu = run_gpu(torch, th, grads, hp, steps=4)
+    # lambda_out is written on root steps only
+    assert np.array_equal(gpu["lam"][1], gpu["lam"][0]) and np.array_equal(gpu["lam"][3], gpu["lam"][2])
+    assert not np.array_equal(gpu["lam"][2], gpu["lam"][0])
+    compare(gpu, th, grads, hp, steps=4)
+
+
+def test_frobenius_scaling_step(torch):
+    shapes = [(256, 384)]
+    grads = [[g] for g in workloads.gaussian_gradients(shapes, std=0.1, seed=22)]
+    th = workloads.parameters(shapes, seed=23)
+    hp = ostep.HParams(block_size=128, ndb_iters1=18, ndb_iters2=16, eps=1e-4, scaling="frobenius")
+    gpu = run_gpu(torch, th, grads, hp)
+    # lambda = ||L + eps I||_F of each step-1 factor
+    f = 0
+    G = grads[0][0].astype(np.float32).astype(np.float64)
+    for (r0, r1, c0, c1) in ostep.block_grid(*G.shape, 128):
+        Gb = G[r0:r1, c0:c1]
+        for A in (Gb @ Gb.T, Gb.T @ Gb):
+            Ab = hp.beta * hp.init_scale * np.eye(A.shape[0]) + (1 - hp.beta) * A + hp.eps * np.eye(A.shape[0])
+            ref = np.linalg.norm(Ab, "fro")
+            assert abs(gpu["lam"][0][f] - ref) <= 1e-5 * ref, (f, gpu["lam"][0][f], ref)
+            f += 1
+    compare(gpu, th, grads, hp)

@@ -164,3 +164,42 @@ def test_first_step_block_update_matches_full_step():
         d, _, s = step.first_step_block_update(G[r0:r1, c0:c1], info["P"][0][r0:r1, c0:c1], hp,
                                                info["lam"][2 * k], info["lam"][2 * k + 1])
         assert rel(d, new[0][r0:r1, c0:c1]) < 1e-13 and s == pytest.approx(info["graft"][k], rel=1e-13)
+
+
+def test_frobenius_scale_is_the_frobenius_norm_diagonal():
+    # diagonal factor: ||A||_F = sqrt(sum lambda_i^2), an upper bound of
+    # lambda_max; with enough iterations the truncated root at that scale is
+    # the exact diag(lambda^-1/4)
+    lam = np.array([3.0, 1.0, 0.5, 0.25, 0.1, 0.05, 0.02, 0.01])
+    A = np.diag(lam)
+    hp = step.HParams(block_size=8, scaling="frobenius", ndb_iters1=40, ndb_iters2=40, root_level=2)
+    X, lam_est = step.inverse_fourth_root(A, None, hp)
+    assert lam_est == pytest.approx(np.sqrt(np.sum(lam ** 2)), rel=1e-15)
+    assert lam_est >= lam.max()
+    assert rel(X, np.diag(lam ** -0.25)) < 1e-10
+    hp.scaling = "nonsense"
+    with pytest.raises(ValueError):
+        step.inverse_fourth_root(A, None, hp)
+
+
+def test_root_every_reuses_the_last_root_step_closed_form():
+    # gradients sigma_t Q_t with Q_t orthogonal keep every factor a multiple of
+    # I: after step t, L = R = a_t I with a_t = beta a_{t-1} + (1-beta) sigma_t^2,
+    # a_0 = init_scale.  Exact roots (level 1) give U_t = sigma_t Q_t (a + eps)^-1/2
+    # where a is a_t on root steps and the last root step's a otherwise.
+    rng = np.random.default_rng(7)
+    b, sig = 8, [0.7, 1.9, 0.4, 1.1]
+    Qs = [workloads.haar_orthogonal(b, rng) for _ in sig]
+    V0 = workloads.pi_start_vectors(b, 32, seed=0)
+    for every, roots_at in [(1, [1, 2, 3, 4]), (2, [1, 3]), (3, [1, 4])]:
+        hp = step.HParams(block_size=b, root_level=1, root_every=every)
+        state = step.init_state([(b, b)], hp)
+        th = [np.zeros((b, b))]
+        a, a_root = hp.init_scale, None
+        for t, (s_t, Q) in enumerate(zip(sig, Qs), start=1):
+            th, state, info = step.shampoo_step(th, [s_t * Q], state, hp, V0)
+            a = hp.beta * a + (1 - hp.beta) * s_t ** 2
+            if t in roots_at:
+                a_root = a
+            assert info["root_step"] == (t in roots_at)
+            assert rel(info["U"][0], s_t * Q * (a_root + hp.eps) ** -0.5) < 1e-12

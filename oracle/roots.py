@@ -141,6 +141,62 @@ def ndb_inv4root_matmul(A, lam_est, iters1, iters2):
 
 
 # --------------------------------------------------------------------------
+# Coupled Newton
+# --------------------------------------------------------------------------
+
+def cn_scalar(m0, iters, p=4):
+    """The coupled-Newton recurrence on scalars (element-wise on arrays).
+
+    DASH explainer, "Building blocks" (Coupled-Newton): X_k ~ A^(-1/p) with a
+    stabiliser M_k; C_k is computed from M_k, X_{k+1} = X_k C_k and
+    M_{k+1} = C_k^p M_k.  Reading for the unstated C_k: the Newton step
+    C_k = ((p+1) - M_k)/p.  From x0 = 1, m0 = c*w: x -> m0^(-1/p) for
+    0 < m0 < p+1, and m = x^p * m0 at every step.  Returns (x, m).
+    """
+    m = np.array(m0, dtype=np.float64, copy=True)
+    x = np.ones_like(m)
+    for _ in range(iters):
+        c = ((p + 1.0) - m) / p
+        x, m = x * c, c ** p * m
+    return x, m
+
+
+def cn_phi(w, lam_est, iters):
+    """Scalar map of the coupled-Newton inverse fourth root: the common
+    scaling c = 1/(2 lambda_est), M0 = c w, X0 = 1, result c^(1/4) x."""
+    c = ndb_scale(lam_est)
+    x, _ = cn_scalar(c * np.asarray(w, dtype=np.float64), iters)
+    return c ** 0.25 * x
+
+
+def cn_inv4root_spectral(A, lam_est, iters):
+    """Level 2: the truncated coupled-Newton result, evaluated exactly."""
+    A = np.asarray(A, dtype=np.float64)
+    w, Q = np.linalg.eigh(0.5 * (A + A.T))
+    return (Q * cn_phi(w, lam_est, iters)) @ Q.T
+
+
+def cn_matrix(M0, iters, p=4):
+    """Coupled Newton with matrices, step by step (level 3), from X0 = I:
+    C = ((p+1) I - M)/p; X <- X C; M <- C^p M."""
+    M = np.array(M0, dtype=np.float64, copy=True)
+    I = np.eye(M.shape[0])
+    X = I.copy()
+    for _ in range(iters):
+        C = ((p + 1.0) * I - M) / p
+        X, M = X @ C, np.linalg.matrix_power(C, p) @ M
+    return X, M
+
+
+def cn_inv4root_matmul(A, lam_est, iters):
+    """Level 3: coupled-Newton inverse fourth root with matrix products,
+    M0 = c A, X0 = I, X = c^(1/4) X_T."""
+    c = ndb_scale(lam_est)
+    X, _ = cn_matrix(c * np.asarray(A, dtype=np.float64), iters)
+    return c ** 0.25 * X
+
+
+# --------------------------------------------------------------------------
 # Chebyshev / Clenshaw
 # --------------------------------------------------------------------------
 

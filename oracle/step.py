@@ -27,7 +27,8 @@ class HParams:
     init_scale=1e-6, textbook bias-corrected Adam (beta1=0.9, beta2=0.999,
     adam_eps=1e-8), per-block grafting, power iteration with ``pi_iters``
     products, Newton-DB ``ndb_iters1`` + ``ndb_iters2`` iterations, Chebyshev
-    degree ``cheb_degree`` on [cheb_delta, 1 + cheb_delta].
+    degree ``cheb_degree`` on [cheb_delta, 1 + cheb_delta], coupled Newton
+    ``cn_iters`` iterations.
 
     ``scaling``: the scale estimate of each factor ("Building blocks",
     scaling): "spectral" (multi-start power iteration) or "frobenius"
@@ -44,11 +45,12 @@ class HParams:
     beta2: float = 0.999
     adam_eps: float = 1e-8
     lr: float = 1e-3
-    solver: str = "ndb"          # "ndb" | "cheb"
+    solver: str = "ndb"          # "ndb" | "cheb" | "cn"
     ndb_iters1: int = 14
     ndb_iters2: int = 14
     cheb_degree: int = 16
     cheb_delta: float = 1e-3
+    cn_iters: int = 16
     pi_iters: int = 10
     root_level: int = 2          # 1 exact, 2 truncated method (spectral), 3 matmul
     scaling: str = "spectral"    # "spectral" | "frobenius"
@@ -103,6 +105,13 @@ def inverse_fourth_root(Abar, V0, hp, lam_est=None):
             X = roots.ndb_inv4root_spectral(Abar, lam_est, hp.ndb_iters1, hp.ndb_iters2)
         else:
             X = roots.ndb_inv4root_matmul(Abar, lam_est, hp.ndb_iters1, hp.ndb_iters2)
+    elif hp.solver == "cn":
+        if hp.root_level == 1:
+            X = roots.inv_root_eigh(Abar, 4)
+        elif hp.root_level == 2:
+            X = roots.cn_inv4root_spectral(Abar, lam_est, hp.cn_iters)
+        else:
+            X = roots.cn_inv4root_matmul(Abar, lam_est, hp.cn_iters)
     elif hp.solver == "cheb":
         if hp.root_level == 1:
             shift = hp.cheb_delta / roots.ndb_scale(lam_est)

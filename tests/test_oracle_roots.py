@@ -167,6 +167,51 @@ def test_ndb_config2_convergence_profile():
     assert np.max(np.abs(phi8 / lam ** -0.25 - 1.0)) > 1e-2
 
 
+# ---------------------------------------------------------------- coupled Newton
+
+
+@pytest.mark.parametrize("iters", [0, 1, 4, 12])
+def test_cn_scalar_keeps_the_coupling_invariant(iters):
+    # every coupled-Newton step keeps m = x^4 * m0 (C multiplies x once and
+    # m four times), so a wrong power or a dropped factor breaks it
+    m0 = np.geomspace(1e-6, 4.9, 60)
+    x, m = roots.cn_scalar(m0, iters)
+    assert np.allclose(m, x ** 4 * m0, rtol=1e-12, atol=0)
+
+
+def test_cn_scalar_converges_to_inverse_fourth_root():
+    m0 = np.geomspace(1e-6, 4.5, 60)
+    x, m = roots.cn_scalar(m0, 60)
+    assert np.max(np.abs(x / m0 ** -0.25 - 1.0)) < 1e-12
+    assert np.max(np.abs(m - 1.0)) < 1e-12
+    # outside (0, p + 1) = (0, 5) the iteration leaves the basin
+    x, _ = roots.cn_scalar(np.array([5.5]), 30)
+    assert not np.isfinite(x[0]) or abs(x[0] - 5.5 ** -0.25) > 1e-3
+
+
+def test_cn_matrix_keeps_the_coupling_invariant():
+    A, _, w = random_spd(24, 1e2, seed=11)
+    M0 = A / (2.0 * w.max())
+    for T in (1, 3, 6):
+        X, M = roots.cn_matrix(M0, T)
+        assert rel(M, np.linalg.matrix_power(X, 4) @ M0) < 1e-12
+
+
+def test_cn_level2_matches_level3():
+    A, _, w = random_spd(48, 1e3, seed=12)
+    lam = w.max() * 0.999
+    for T in (3, 9, 16):
+        assert rel(roots.cn_inv4root_spectral(A, lam, T), roots.cn_inv4root_matmul(A, lam, T)) < 1e-10
+
+
+def test_cn_converges_to_exact():
+    A, _, w = random_spd(48, 1e3, seed=13)
+    assert rel(roots.cn_inv4root_spectral(A, w.max(), 30), roots.inv_root_eigh(A)) < 1e-10
+    # identity: lambda_est = alpha exactly, M0 = 1/2 I, X -> alpha^(-1/4) I
+    X = roots.cn_inv4root_matmul(3.0 * np.eye(5), 3.0, 25)
+    assert rel(X, 3.0 ** -0.25 * np.eye(5)) < 1e-12
+
+
 # ---------------------------------------------------------------- Chebyshev
 
 @pytest.mark.parametrize("degree,delta", [(4, 0.1), (16, 1e-3), (16, 1e-6), (60, 1e-3)])

@@ -50,7 +50,9 @@ def parse_args():
     p.add_argument("--workload", default="llama1b",
                    choices=["llama1b", "gpt2", "spiked512", "roots256", "mixed"])
     p.add_argument("--block", type=int, default=None, help="override the block size")
-    p.add_argument("--solver", default="ndb", choices=["ndb", "cheb"])
+    p.add_argument("--solver", default="ndb", choices=["ndb", "cheb", "cn", "cn16"],
+                   help="Newton-DB, Chebyshev, coupled Newton (split products) or coupled Newton in fp16")
+    p.add_argument("--cn-iters", type=int, default=16)
     p.add_argument("--iters", type=int, default=None, help="Newton-DB iterations per stage")
     p.add_argument("--degree", type=int, default=16)
     p.add_argument("--n", type=int, default=256, help="matrices in the standalone-roots workload")
@@ -184,7 +186,8 @@ def oracle_sample(spec, args, budget_s=15.0, seed=0):
     B = spec["B"]
     iters = spec["iters"]
     hp = ostep.HParams(block_size=B, ndb_iters1=iters, ndb_iters2=iters,
-                       solver="ndb" if args.solver == "ndb" else "cheb", cheb_degree=args.degree)
+                       solver={"ndb": "ndb", "cheb": "cheb"}.get(args.solver, "cn"), cheb_degree=args.degree,
+                       cn_iters=args.cn_iters)
     V0 = wl.pi_start_vectors(B, 32, seed=0).astype(np.float64)
     if spec["shapes"] is None:  # standalone roots: time per matrix
         nmat = spec.get("n", 256)
@@ -192,8 +195,7 @@ def oracle_sample(spec, args, budget_s=15.0, seed=0):
         t0 = time.perf_counter()
         done = 0
         for i in range(A.shape[0]):
-            lam, _ = roots.power_iteration(A[i].astype(np.float64), V0, 10)
-            roots.ndb_inv4root_spectral(A[i].astype(np.float64), lam, iters, iters)
+            ostep.inverse_fourth_root(A[i].astype(np.float64), V0, hp)  # power iteration + the solver
             done += 1
             if time.perf_counter() - t0 > budget_s:
                 break
@@ -279,7 +281,8 @@ def main():
 
     B = spec["B"]
     iters = spec["iters"]
-    solver = bd.SOLVER_NEWTON_DB if args.solver == "ndb" else bd.SOLVER_CHEBYSHEV
+    solver = {"ndb": bd.SOLVER_NEWTON_DB, "cheb": bd.SOLVER_CHEBYSHEV}.get(args.solver, bd.SOLVER_COUPLED_NEWTON)
+    cn16 = args.solver == "cn16"
     stream = torch.cuda.current_stream()
 
     if spec["shapes"] is None:
@@ -296,6 +299,8 @@ def main():
         def step_fn():
             if solver == bd.SOLVER_NEWTON_DB:
                 bd.inv_root_newton_db(At, v0, iters, iters, 0.0, 10, X, lam, ws)
+            elif solver == bd.SOLVER_COUPLED_NEWTON:
+                bd.inv_root_coupled_newton(At, v0, args.cn_iters, cn16, 0.0, 10, X, lam, ws)
             else:
                 bd.inv_root_chebyshev(At, v0, args.degree, 1e-3, 0.0, 10, X, lam, ws)
         n_factors, factor_sizes = nmat, [B] * nmat
@@ -305,7 +310,8 @@ def main():
         grads = make_grads(spec, dev, seed=0)
         params = [torch.randn(g.shape, device=dev) * 0.02 for g in grads]
         hp = bd.make_hparams(block_size=B, solver=solver, ndb_iters1=iters, ndb_iters2=iters,
-                             cheb_degree=args.degree, root_every=args.root_every,
+                             cheb_degree=args.degree, root_every=args.root_every, cn_iters=args.cn_iters,
+                             cn_fp16=1 if cn16 else 0,
                              scaling=bd.SCALING_FROBENIUS if args.scaling == "frobenius" else bd.SCALING_SPECTRAL)
         opt = bd.Shampoo(params, grads, hp=hp,
                          v0=torch.from_numpy(wl.pi_start_vectors(B, 32, seed=0)).to(dev))
@@ -409,8 +415,8 @@ def main():
     g_ms, g_n, g_flops = prof["gemm"]
     tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     avg_ms = g_ms / max(g_n, 1)
-    # 3 fp16 MMA products (hi*hi, hi*lo, lo*hi) per useful product
-    achieved = 3.0 * (g_flops / max(g_n, 1)) / (avg_ms * 1e-3) / 1e12 if g_n else None
+    # executed fp16 MMA flops as the library records them (3 per useful product, 1 in fp16 mode)
+    achieved = (g_flops / max(g_n, 1)) / (avg_ms * 1e-3) / 1e12 if g_n else None
     roofline = {"kernel": "gemm_split_kernel", "bound": "tensor",
                 "achieved": round(achieved, 1) if achieved else None, "peak": tensor_peak,
                 "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4) if achieved else None,
@@ -422,6 +428,8 @@ def main():
     s_ms = prof["solver"][0] + prof["power_iteration"][0]
     if args.solver == "ndb":
         gemms = 2 * (3 * iters - 3)            # both stages, first-iteration and last-iteration savings
+    elif args.solver in ("cn", "cn16"):
+        gemms = 4 * (args.cn_iters - 1) + 1    # C^2, C^4, C^4 M, X C; the last iteration only X C
     else:
         gemms = args.degree - 1
     padded = 2.0 * B ** 3 * gemms * n_factors
@@ -454,6 +462,7 @@ def main():
             "config": dict({"workload": spec["desc"], "block_size": B, "solver": args.solver,
                             "iters_per_stage": iters if args.solver == "ndb" else None,
                             "cheb_degree": args.degree if args.solver == "cheb" else None,
+                            "cn_iters": args.cn_iters if args.solver in ("cn", "cn16") else None,
                             "scale_estimate": ("power iteration, 10 products x 32 starts" if args.scaling == "spectral"
                                                else "Frobenius norm"),
                             "roots_every_steps": max(1, args.root_every),

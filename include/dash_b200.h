@@ -60,6 +60,7 @@ extern "C" {
 
 #define SHAMPOO_SOLVER_NEWTON_DB 0
 #define SHAMPOO_SOLVER_CHEBYSHEV 1
+#define SHAMPOO_SOLVER_COUPLED_NEWTON 2
 
 /* Scale estimate lambda each factor is divided by (c = 1 / (2 lambda)) before
  * the root solver ("Building blocks", scaling): the multi-start power
@@ -102,6 +103,8 @@ typedef struct {
   int root_every;   /* roots recomputed every root_every-th step (steps 1, 1 + f, ...);
                        other steps reuse the roots kept in the workspace (0 or 1: every step) */
   int scaling;      /* SHAMPOO_SCALING_* */
+  int cn_iters;     /* coupled-Newton iterations, 0..1000 */
+  int cn_fp16;      /* 1: coupled Newton with single-pass fp16 products (0: fp32-level split products) */
 } shampoo_hparams;
 
 /* Build the block table for a parameter set (host only; no device work).
@@ -140,7 +143,7 @@ SHAMPOO_API int shampoo_accumulate(shampoo_ctx* ctx, float* factors, void* ws, s
  * flow" after the EMA; "Step-by-step" steps "Scale each block",
  * "Compute inverse roots", "Grafting with Adam's magnitude", "Apply update"):
  *   for every factor F: A = F + eps I; lambda = power iteration on A from v0;
- *   X = A^(-1/4) by the configured solver (Newton-DB or Chebyshev, as for the
+ *   X = A^(-1/4) by the configured solver (Newton-DB, Chebyshev or coupled Newton, as for the
  *   standalone calls below); then per block U = X_L G X_R; Adam moments
  *   m, v (bias-corrected with `step` >= 1); P = m_hat / (sqrt(v_hat) + adam_eps);
  *   s = ||P_b||_F / ||U_b||_F (0 when U_b = 0); param -= lr * s * U_b.
@@ -182,6 +185,19 @@ SHAMPOO_API int shampoo_inv_root_newton_db(const float* A, float* X, int n, int 
 SHAMPOO_API int shampoo_inv_root_chebyshev(const float* A, float* X, int n, int B, int degree, float delta, float eps,
                                const float* v0, int pi_iters, float* lambda_out, void* ws, size_t ws_bytes,
                                void* stream);
+
+/* Standalone inverse fourth roots of a stack, coupled-Newton solver
+ * ("Building blocks", Coupled-Newton; "Scoreboard": CN in FP16):
+ *   A_i' = A_i + eps I;  lambda_i as for the Newton-DB call;  c = 1/(2 lambda_i);
+ *   M = c A_i', X = I;  `iters` times: C = (5I - M)/4, X <- X C, M <- C^4 M;
+ *   X_i = c^(1/4) X  ~  (A_i + eps I)^(-1/4).
+ * fp16 = 1 computes every product in one pass of fp16 operands with fp32
+ * accumulation (the pages' fast mode); fp16 = 0 uses the split-fp16 products
+ * of the other solvers (about fp32 accuracy).  Other arguments as for the
+ * Newton-DB call. */
+SHAMPOO_API int shampoo_inv_root_coupled_newton(const float* A, float* X, int n, int B, int iters, int fp16,
+                                                float eps, const float* v0, int pi_iters, float* lambda_out,
+                                                void* ws, size_t ws_bytes, void* stream);
 
 /* Variant of shampoo_inv_root_newton_db that allocates nothing and needs no
  * workspace from the caller.  The paper has no counterpart: this exists for
@@ -233,8 +249,9 @@ SHAMPOO_API int shampoo_profile_enable(int enable);
 /* Forget everything recorded so far. */
 SHAMPOO_API int shampoo_profile_reset(void);
 /* Synchronise the recorded events and fill out[0 .. 19] (n >= 20):
- * out[3s], out[3s+1], out[3s+2] = milliseconds, count and useful flops of
- * stage s, for s = 0 GEMM launches (flops = 2*128*128*B per computed tile),
+ * out[3s], out[3s+1], out[3s+2] = milliseconds, count and flops of stage s,
+ * for s = 0 GEMM launches (executed tensor-core flops: 3 * 2*128*128*B per
+ * computed tile, or 1 * ... for single-pass fp16 launches),
  * 1 gather + factor EMA, 2 power iteration, 3 root solver, 4 preconditioner
  * products, 5 Adam graft + update; out[18] = kernel launches since the last
  * reset; out[19] = records dropped. */

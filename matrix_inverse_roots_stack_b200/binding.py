@@ -22,6 +22,7 @@ SHAMPOO_ENONFINITE = -5
 SHAMPOO_ETIMEOUT = -6
 SOLVER_NEWTON_DB = 0
 SOLVER_CHEBYSHEV = 1
+SOLVER_COUPLED_NEWTON = 2
 SCALING_SPECTRAL = 0
 SCALING_FROBENIUS = 1
 PI_STARTS = 32
@@ -44,16 +45,17 @@ class ShampooHParams(ctypes.Structure):
                 ("adam_eps", ctypes.c_float), ("lr", ctypes.c_float), ("solver", ctypes.c_int),
                 ("ndb_iters1", ctypes.c_int), ("ndb_iters2", ctypes.c_int), ("cheb_degree", ctypes.c_int),
                 ("cheb_delta", ctypes.c_float), ("pi_starts", ctypes.c_int), ("pi_iters", ctypes.c_int),
-                ("root_every", ctypes.c_int), ("scaling", ctypes.c_int)]
+                ("root_every", ctypes.c_int), ("scaling", ctypes.c_int), ("cn_iters", ctypes.c_int),
+                ("cn_fp16", ctypes.c_int)]
 
 
 def make_hparams(block_size=1024, beta=0.95, eps=1e-6, init_scale=1e-6, beta1=0.9, beta2=0.999,
                  adam_eps=1e-8, lr=1e-3, solver=SOLVER_NEWTON_DB, ndb_iters1=14, ndb_iters2=14,
                  cheb_degree=16, cheb_delta=1e-3, pi_starts=PI_STARTS, pi_iters=10, root_every=1,
-                 scaling=SCALING_SPECTRAL):
+                 scaling=SCALING_SPECTRAL, cn_iters=16, cn_fp16=0):
     return ShampooHParams(block_size, beta, eps, init_scale, beta1, beta2, adam_eps, lr, solver,
                           ndb_iters1, ndb_iters2, cheb_degree, cheb_delta, pi_starts, pi_iters, root_every,
-                          scaling)
+                          scaling, cn_iters, cn_fp16)
 
 
 _lib = None
@@ -69,6 +71,7 @@ _PROTOS = {
     "shampoo_precondition_step": (_I, [_VP, _VP, _VP, _I, _VP, _VP, _VP, _SZ, _VP]),
     "shampoo_inv_root_newton_db": (_I, [_VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _VP, _VP, _SZ, _VP]),
     "shampoo_inv_root_chebyshev": (_I, [_VP, _VP, _I, _I, _I, _F, _F, _VP, _I, _VP, _VP, _SZ, _VP]),
+    "shampoo_inv_root_coupled_newton": (_I, [_VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _VP, _VP, _SZ, _VP]),
     "shampoo_inv_root_workspace_bytes": (_SZ, [_I, _I, _I]),
     "shampoo_read_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_uint)]),
     "shampoo_strerror": (ctypes.c_char_p, [_I]),
@@ -167,6 +170,22 @@ def inv_root_chebyshev(A, v0, degree=16, delta=1e-3, eps=0.0, pi_iters=10, X=Non
 
 
 STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def inv_root_coupled_newton(A, v0, iters=16, fp16=False, eps=0.0, pi_iters=10, X=None, lam=None, ws=None,
+                            stream=None):
+    """Coupled-Newton variant of :func:`inv_root_newton_db` (fp16: single-pass
+    fp16 products)."""
+    import torch
+    n, B = A.shape[0], A.shape[1]
+    X = torch.empty_like(A) if X is None else X
+    lam = torch.empty(n, dtype=torch.float32, device=A.device) if lam is None else lam
+    need = inv_root_workspace_bytes(n, B, SOLVER_COUPLED_NEWTON)
+    ws = _workspace(need, A.device) if ws is None else ws
+    rc = load().shampoo_inv_root_coupled_newton(_ptr(A), _ptr(X), n, B, iters, 1 if fp16 else 0, eps, _ptr(v0),
+                                                pi_iters, _ptr(lam), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "shampoo_inv_root_coupled_newton")
+    return X, lam, ws
 
 
 def inv_root_newton_db_static(A, v0, iters1=14, iters2=14, eps=0.0, pi_iters=10, X=None, lam=None, stream=None):

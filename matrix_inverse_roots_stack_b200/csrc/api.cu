@@ -37,11 +37,14 @@ struct Bump {
   }
 };
 
-// Factors per solver chunk: the Newton-DB scratch is 5 split matrices per
-// factor (Chebyshev needs 4), bounded by kSolverBudget.
-constexpr int kSolverMats = 5;
-int solver_chunk(int nf, int B) {
-  const size_t per = kSolverMats * split_bytes(1, B);
+// Split matrices of solver scratch per factor: Newton-DB 5 (Y and Z
+// ping-pong, D), Chebyshev 4 (T and the Clenshaw ring), coupled Newton 6 (M
+// and X ping-pong, C^2, C^4).  Chunks of factors keep it within kSolverBudget.
+int solver_mats(int solver) {
+  return solver == SHAMPOO_SOLVER_COUPLED_NEWTON ? 6 : solver == SHAMPOO_SOLVER_CHEBYSHEV ? 4 : 5;
+}
+int solver_chunk(int nf, int B, int solver) {
+  const size_t per = solver_mats(solver) * split_bytes(1, B);
   size_t m = kSolverBudget / per;
   if (m < 1) m = 1;
   return static_cast<int>(m < static_cast<size_t>(nf) ? m : nf);
@@ -53,15 +56,16 @@ struct RootLayout {
   int chunk;
 };
 
-void plan_roots(Bump& b, RootLayout& L, int nf, int B, int pi_iters, int extra_mats) {
+void plan_roots(Bump& b, RootLayout& L, int nf, int B, int pi_iters, int extra_mats, int solver) {
   L.status = b.take(256);
   L.lam = b.take(sizeof(float) * nf);
   L.xscale = b.take(sizeof(float) * nf);
   L.stats = b.take(sizeof(float) * static_cast<size_t>(pi_iters) * nf * 3 * dash::kPiStarts);
   L.w0 = b.take(sizeof(float) * static_cast<size_t>(nf) * B * dash::kPiStarts);
   L.w1 = b.take(sizeof(float) * static_cast<size_t>(nf) * B * dash::kPiStarts);
-  L.chunk = solver_chunk(nf, B);
-  const int mats = kSolverMats * L.chunk > extra_mats ? kSolverMats * L.chunk : extra_mats;
+  L.chunk = solver_chunk(nf, B, solver);
+  const int per = solver_mats(solver);
+  const int mats = per * L.chunk > extra_mats ? per * L.chunk : extra_mats;
   L.solver = b.take(split_bytes(mats, B));
 }
 
@@ -291,8 +295,96 @@ int run_cheb_chunk(const float* F, int n, int B, float eps, const int* fsize, co
   return SHAMPOO_OK;
 }
 
-// Power iteration + solver on nf factors.  Writes X as fp32 (X_f32) and/or
-// split (X_split).  fsize (device) gives each factor's true size or is null.
+// Coupled Newton on one chunk of n factors ("Building blocks", Coupled-Newton:
+// C_k from M_k; X_{k+1} = X_k C_k; M_{k+1} = C_k^p M_k; C_k = (5I - M_k)/4 for
+// p = 4).  Every iterate is a polynomial in A, so each product is symmetric
+// and computed on upper-triangle tiles (mirrored); the iteration for M is a
+// function of M alone, so symmetrising it is harmless.  Per iteration:
+//   C^2 = (M M - 10 M + 25 I)/16;  C^4 = C^2 C^2;
+//   M' = C^4 M  and  X' = (5 X - X M)/4  (one launch, both read the old M);
+// the last iteration needs only X'.  fp16: single-pass fp16 products.
+int run_cn_chunk(const float* F, int n, int B, float eps, const int* fsize, const float* lam, float* xscale,
+                 int iters, int fp16, float* X_f32, __half* X_split, __half* S, unsigned* status,
+                 cudaStream_t st) {
+  const size_t m = static_cast<size_t>(n) * 2 * B * B;
+  __half* Mb[2] = {S, S + m};
+  __half* Xb[2] = {S + 2 * m, S + 3 * m};
+  __half* C2 = S + 4 * m;
+  __half* C4 = S + 5 * m;
+  int mc = 0, xc = 0;
+  dash::launch_cn_init(F, n, B, eps, fsize, lam, Mb[0], Xb[0], xscale, st);
+  DASH_LAUNCHED();
+  if (iters == 0) {
+    dash::launch_scale_split(Xb[0], n, B, xscale, X_f32, X_split, st);
+    DASH_LAUNCHED();
+    return SHAMPOO_OK;
+  }
+  auto base = [&]() {
+    GemmArgs g = gemm_args(B, 1, status);
+    g.single_pass = fp16 ? 1 : 0;
+    g.op[0].nprob = n;
+    return g;
+  };
+  for (int it = 0; it < iters; ++it) {
+    const bool last = it == iters - 1;
+    if (!last) {
+      {  // C^2 = M M / 16 - (10/16) M + (25/16) I
+        GemmArgs g = base();
+        dash::GemmOp& o = g.op[0];
+        o.alpha = 1.0f / 16.0f;
+        o.beta = -10.0f / 16.0f;
+        o.cin_split = Mb[mc];
+        o.gamma = 25.0f / 16.0f;
+        o.out_split = C2;
+        dash::OpBuffers ob[2] = {{Mb[mc], n, Mb[mc], n}, {Mb[mc], n, Mb[mc], n}};
+        DASH_TRY(dash::launch_gemm_split(ob, g, st));
+      }
+      {  // C^4 = C^2 C^2
+        GemmArgs g = base();
+        dash::GemmOp& o = g.op[0];
+        o.alpha = 1.0f;
+        o.out_split = C4;
+        dash::OpBuffers ob[2] = {{C2, n, C2, n}, {C2, n, C2, n}};
+        DASH_TRY(dash::launch_gemm_split(ob, g, st));
+      }
+    }
+    GemmArgs g = base();
+    dash::OpBuffers ob[2];
+    int xo = 0;
+    if (!last) {  // M' = C^4 M
+      dash::GemmOp& o = g.op[0];
+      o.alpha = 1.0f;
+      o.out_split = Mb[mc ^ 1];
+      ob[0] = {C4, n, Mb[mc], n};
+      g.op[1].nprob = n;
+      g.nops = 2;
+      xo = 1;
+    }
+    {  // X' = (5 X - X M)/4, scaled by c^(1/4) into the outputs on the last iteration
+      dash::GemmOp& o = g.op[xo];
+      o.alpha = -0.25f;
+      o.beta = 1.25f;
+      o.cin_split = Xb[xc];
+      if (last) {
+        o.out_split = X_split;
+        o.out_f32 = X_f32;
+        o.scale = xscale;
+      } else {
+        o.out_split = Xb[xc ^ 1];
+      }
+      ob[xo] = {Xb[xc], n, Mb[mc], n};
+    }
+    DASH_TRY(dash::launch_gemm_split(ob, g, st));
+    mc ^= 1;
+    xc ^= 1;
+  }
+  return SHAMPOO_OK;
+}
+
+// Power iteration (pi_iters > 0) or Frobenius norm (pi_iters == 0) + solver
+// on nf factors.  Writes X as fp32 (X_f32) and/or split (X_split).  fsize
+// (device) gives each factor's true size or is null.  it1, it2: the Newton-DB
+// stage iterations, or for the coupled Newton its iterations and fp16 flag.
 int run_roots(const float* F, int nf, int B, float eps, const int* fsize, const float* v0, int pi_iters, int solver,
               int it1, int it2, int degree, float delta, float* lam_out, float* X_f32, __half* X_split, char* ws,
               const RootLayout& L, unsigned* status, cudaStream_t st) {
@@ -329,10 +421,12 @@ int run_roots(const float* F, int nf, int B, float eps, const int* fsize, const 
     const int* fs = fsize ? fsize + f0 : nullptr;
     float* Xf = X_f32 ? X_f32 + f0 * BB : nullptr;
     __half* Xs = X_split ? X_split + f0 * 2 * BB : nullptr;
-    const int rc = (solver == SHAMPOO_SOLVER_NEWTON_DB)
-                       ? run_ndb_chunk(Fc, n, B, eps, fs, lam + f0, xscale + f0, it1, it2, Xf, Xs, S, status, st)
-                       : run_cheb_chunk(Fc, n, B, eps, fs, lam + f0, xscale + f0, degree, c, Xf, Xs, S, status,
-                                        st);
+    const int rc =
+        (solver == SHAMPOO_SOLVER_NEWTON_DB)
+            ? run_ndb_chunk(Fc, n, B, eps, fs, lam + f0, xscale + f0, it1, it2, Xf, Xs, S, status, st)
+        : (solver == SHAMPOO_SOLVER_COUPLED_NEWTON)
+            ? run_cn_chunk(Fc, n, B, eps, fs, lam + f0, xscale + f0, it1, it2, Xf, Xs, S, status, st)
+            : run_cheb_chunk(Fc, n, B, eps, fs, lam + f0, xscale + f0, degree, c, Xf, Xs, S, status, st);
     if (rc) {
       dash::prof_end(sslot, st);
       return rc;
@@ -394,7 +488,10 @@ int check_hparams(const shampoo_hparams* hp) {
   if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
       !finite_nonneg(hp->adam_eps) || !std::isfinite(hp->lr))
     return SHAMPOO_EINVAL;
-  if (hp->solver != SHAMPOO_SOLVER_NEWTON_DB && hp->solver != SHAMPOO_SOLVER_CHEBYSHEV) return SHAMPOO_EINVAL;
+  if (hp->solver != SHAMPOO_SOLVER_NEWTON_DB && hp->solver != SHAMPOO_SOLVER_CHEBYSHEV &&
+      hp->solver != SHAMPOO_SOLVER_COUPLED_NEWTON)
+    return SHAMPOO_EINVAL;
+  if (hp->cn_iters < 0 || hp->cn_iters > 1000 || (hp->cn_fp16 != 0 && hp->cn_fp16 != 1)) return SHAMPOO_EINVAL;
   if (hp->ndb_iters1 < 1 || hp->ndb_iters2 < 1 || hp->ndb_iters1 > 1000 || hp->ndb_iters2 > 1000)
     return SHAMPOO_EINVAL;
   if (hp->cheb_degree < 2 || hp->cheb_degree > 256 || !(hp->cheb_delta > 0.0f) || !std::isfinite(hp->cheb_delta))
@@ -473,7 +570,7 @@ int shampoo_init_blocks(shampoo_ctx** out, const shampoo_param* params, int n_pa
     return SHAMPOO_EUNSUPPORTED;
   }
   Bump b;
-  plan_roots(b, c->roots, c->n_factors, B, hp->pi_iters, c->n_blocks);
+  plan_roots(b, c->roots, c->n_factors, B, hp->pi_iters, c->n_blocks, hp->solver);
   c->off_gs = b.take(split_bytes(c->n_factors, B));
   c->off_roots = b.take(split_bytes(c->n_factors, B));
   c->off_u = b.take(sizeof(float) * static_cast<size_t>(c->total_elems));
@@ -568,8 +665,10 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   const int every = hp.root_every > 0 ? hp.root_every : 1;
   if ((step - 1) % every == 0 || ctx->roots_ws != ws_v) {  // root step (or no roots kept in this ws yet)
     const int pi = hp.scaling == SHAMPOO_SCALING_FROBENIUS ? 0 : hp.pi_iters;
-    rc = run_roots(factors, nf, B, hp.eps, fsize, v0, pi, hp.solver, hp.ndb_iters1, hp.ndb_iters2, hp.cheb_degree,
-                   hp.cheb_delta, lambda_out, roots_out, roots, ws, ctx->roots, status, st);
+    const bool cn = hp.solver == SHAMPOO_SOLVER_COUPLED_NEWTON;
+    rc = run_roots(factors, nf, B, hp.eps, fsize, v0, pi, hp.solver, cn ? hp.cn_iters : hp.ndb_iters1,
+                   cn ? hp.cn_fp16 : hp.ndb_iters2, hp.cheb_degree, hp.cheb_delta, lambda_out, roots_out, roots, ws,
+                   ctx->roots, status, st);
     if (rc) return rc;
     ctx->roots_ws = ws_v;
   }
@@ -629,7 +728,7 @@ size_t shampoo_inv_root_workspace_bytes(int n, int B, int solver) {
   if (n < 1 || !valid_B(B)) return 0;
   Bump b;
   RootLayout L;
-  plan_roots(b, L, n, B, 100, 0);
+  plan_roots(b, L, n, B, 100, 0, solver);
   return b.off;
 }
 
@@ -644,7 +743,7 @@ static int inv_root_common(const float* A, float* X, int n, int B, float eps, co
   if (rc) return rc;
   Bump b;
   RootLayout L;
-  plan_roots(b, L, n, B, 100, 0);
+  plan_roots(b, L, n, B, 100, 0, solver);
   char* w = static_cast<char*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned* status = reinterpret_cast<unsigned*>(w + L.status);
@@ -667,6 +766,14 @@ int shampoo_inv_root_chebyshev(const float* A, float* X, int n, int B, int degre
   if (degree < 2 || degree > 256 || !(delta > 0.0f) || !std::isfinite(delta)) return SHAMPOO_EINVAL;
   return inv_root_common(A, X, n, B, eps, v0, pi_iters, ws, ws_bytes, SHAMPOO_SOLVER_CHEBYSHEV, 0, 0, degree, delta,
                          lambda_out, stream);
+}
+
+int shampoo_inv_root_coupled_newton(const float* A, float* X, int n, int B, int iters, int fp16, float eps,
+                                    const float* v0, int pi_iters, float* lambda_out, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  if (iters < 0 || iters > 1000 || (fp16 != 0 && fp16 != 1)) return SHAMPOO_EINVAL;
+  return inv_root_common(A, X, n, B, eps, v0, pi_iters, ws, ws_bytes, SHAMPOO_SOLVER_COUPLED_NEWTON, iters, fp16, 0,
+                         0.0f, lambda_out, stream);
 }
 
 int shampoo_read_status(const void* ws, void* stream, unsigned* flags) {

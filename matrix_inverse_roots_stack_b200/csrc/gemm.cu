@@ -176,6 +176,9 @@ __device__ __forceinline__ void join_chunk(const SplitChunk& c, float* out) {
   }
 }
 
+// kSingle: one pass of hi*hi only (fp16 operands, fp32 accumulation); the lo
+// planes are neither loaded nor multiplied and each K=64 slab is one segment.
+template <bool kSingle>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_split_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                       const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt = args.B / kTile;
   const int tpp = args.sym ? nt * (nt + 1) / 2 : nt * nt;
   const int nk = args.B / kKBlk;
-  const int nsteps = nk * (kKBlk / 16);  // K=16 steps per tile
+  const int nsteps = kSingle ? nk : nk * (kKBlk / 16);  // accumulator segments per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -239,11 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
+          mbar_arrive_expect_tx(&bars->full[s], kSingle ? kStageBytes / 2 : kStageBytes);
           tma_load_3d(st, ta, &bars->full[s], kb * kKBlk, ti * kTile, 2 * am);
-          tma_load_3d(st + kTileBytes, ta, &bars->full[s], kb * kKBlk, ti * kTile, 2 * am + 1);
+          if (!kSingle) tma_load_3d(st + kTileBytes, ta, &bars->full[s], kb * kKBlk, ti * kTile, 2 * am + 1);
 #pragma unroll
-          for (int pl = 0; pl < 2; ++pl) {
+          for (int pl = 0; pl < (kSingle ? 1 : 2); ++pl) {
             uint8_t* dst = st + (2 + pl) * kTileBytes;
             if (g.b_mn) {  // rows kb*64.. of B, columns tj*128.. as two 64-column boxes
               tma_load_3d(dst, tb, &bars->full[s], tj * kTile, kb * kKBlk, 2 * bm + pl);
@@ -290,19 +293,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t so = s * (kStageBytes >> 4);
           const uint64_t ah = kd0 + so, al = ah + kTD, bh = bd0 + so, bl = bh + kTD;
-#pragma unroll
-          for (int kk = 0; kk < kKBlk / 16; ++kk) {
+          if (kSingle) {  // the whole slab into one buffer
             ok = mbar_wait(&bars->acc_empty[hb], (hpar >> hb) & 1u, abort_flag);
             hpar ^= 1u << hb;
             if (!ok) break;
             tc_fence_after();
-            const uint32_t ka = 2u * kk, kbo = bstep * kk;
             const uint32_t d = tbase + hb * 128u;
-            mma_f16_ss(d, ah + ka, bl + kbo, idesc, 0u);         // hi * lo
-            mma_f16_ss(d, al + ka, bh + kbo, idesc, 1u);         // + lo * hi
-            mma_f16_ss_acc_down11(d, ah + ka, bh + kbo, idesc);  // hi * hi + 2^-11 * (...)
+#pragma unroll
+            for (int kk = 0; kk < kKBlk / 16; ++kk)
+              mma_f16_ss(d, ah + 2u * kk, bh + bstep * kk, idesc, kk ? 1u : 0u);
             mma_commit(&bars->acc_full[hb]);
             hb = hb == kRing - 1 ? 0u : hb + 1u;
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kKBlk / 16; ++kk) {
+              ok = mbar_wait(&bars->acc_empty[hb], (hpar >> hb) & 1u, abort_flag);
+              hpar ^= 1u << hb;
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t ka = 2u * kk, kbo = bstep * kk;
+              const uint32_t d = tbase + hb * 128u;
+              mma_f16_ss(d, ah + ka, bl + kbo, idesc, 0u);         // hi * lo
+              mma_f16_ss(d, al + ka, bh + kbo, idesc, 1u);         // + lo * hi
+              mma_f16_ss_acc_down11(d, ah + ka, bh + kbo, idesc);  // hi * hi + 2^-11 * (...)
+              mma_commit(&bars->acc_full[hb]);
+              hb = hb == kRing - 1 ? 0u : hb + 1u;
+            }
           }
           if (!ok) break;
           mma_commit(&bars->empty[s]);
@@ -516,17 +532,21 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
     e = encode_split_stack_map(&maps[2 * o + 1], b.b, a.B, b.b_nmat, a.op[o].b_mn ? 64 : kTile);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = cudaFuncSetAttribute(gemm_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmArgs,
+               const long long) = a.single_pass ? gemm_split_kernel<true> : gemm_split_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long nt = a.B / kTile;
   const long long tpp = a.sym ? nt * (nt + 1) / 2 : nt * nt;
   const long long total = tpp * nprob;
   const long long sms = sm_count();
   const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
-  // useful flops: each computed 128 x 128 tile is one 2*128*128*B product
-  const double flops = 2.0 * kTile * kTile * static_cast<double>(a.B) * static_cast<double>(total);
+  // executed tensor-core flops: each computed 128 x 128 tile is one
+  // 2*128*128*B product, done as three fp16 products (one in single-pass mode)
+  const double flops = (a.single_pass ? 1.0 : 3.0) * 2.0 * kTile * kTile * static_cast<double>(a.B) *
+                       static_cast<double>(total);
   const int slot = prof_begin(kProfGemm, stream, flops);
-  gemm_split_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

@@ -65,6 +65,7 @@ struct GemmArgs {
   int B;      // matrix size; multiple of 128
   int sym;    // 1: symmetric outputs (upper-triangle tiles + mirrored writes)
   int nops;   // 1 or 2
+  int single_pass;  // 1: fp16 operands (hi planes only), one MMA per product, fp32 accumulation
   int skip_loads;  // test hook: the producer issues no loads (bounded waits expire)
   GemmOp op[2];
   unsigned* status;  // device status word (non-finite / timeout bits)

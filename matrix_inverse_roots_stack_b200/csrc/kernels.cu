@@ -326,6 +326,34 @@ __global__ void __launch_bounds__(256) cheb_init_kernel(const float* __restrict_
   store_split4(bdm1 + 2 * f * BB, BB, idx, bb);
 }
 
+// Coupled-Newton prologue ("Building blocks", Coupled-Newton): with the
+// common scaling c = 1/(2 lambda), M0 = c (F + eps I) and X0 = I; padding rows
+// and columns get M0 = I (a fixed point: C = I there).  xscale = c^(1/4).
+__global__ void __launch_bounds__(256) cn_init_kernel(const float* __restrict__ F, int B, float eps,
+                                                      const int* __restrict__ fsize, const float* __restrict__ lam,
+                                                      __half* __restrict__ M0, __half* __restrict__ X0,
+                                                      float* __restrict__ xscale) {
+  const int f = blockIdx.y;
+  const size_t BB = static_cast<size_t>(B) * B;
+  const size_t idx = (static_cast<size_t>(blockIdx.x) * 256 + threadIdx.x) * 4;
+  const int b = fsize ? fsize[f] : B;
+  const float c = 0.5f / lam[f];
+  if (idx == 0) xscale[f] = sqrtf(sqrtf(c));
+  const int r = static_cast<int>(idx / B), col = static_cast<int>(idx % B);
+  const float4 a4 = *reinterpret_cast<const float4*>(F + f * BB + idx);
+  const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+  float m[4], x[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int cc = col + e;
+    const float id = (r == cc) ? 1.0f : 0.0f;
+    m[e] = (r < b && cc < b) ? c * (av[e] + id * eps) : id;
+    x[e] = id;
+  }
+  store_split4(M0 + 2 * f * BB, BB, idx, m);
+  store_split4(X0 + 2 * f * BB, BB, idx, x);
+}
+
 // ------------------------------------------------------------ gather
 
 // grid (B/32, B/32, nb), block (32, 8)
@@ -523,6 +551,13 @@ void launch_cheb_init(const float* F, int nf, int B, float eps, const int* fsize
                       float c_dm1, float c_d, __half* T, __half* bdm1, float* xscale, cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(static_cast<size_t>(B) * B / 1024), nf);
   cheb_init_kernel<<<grid, 256, 0, st>>>(F, B, eps, fsize, lambda, c_dm1, c_d, T, bdm1, xscale);
+  prof_count_launch();
+}
+
+void launch_cn_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, __half* M0,
+                    __half* X0, float* xscale, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>(static_cast<size_t>(B) * B / 1024), nf);
+  cn_init_kernel<<<grid, 256, 0, st>>>(F, B, eps, fsize, lambda, M0, X0, xscale);
   prof_count_launch();
 }
 

@@ -63,6 +63,11 @@ void launch_scale_split(const __half* Z, int nf, int B, const float* xscale, flo
 void launch_cheb_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda,
                       float c_dm1, float c_d, __half* T, __half* bdm1, float* xscale, cudaStream_t st);
 
+// Coupled-Newton prologue: M0 = c (F + eps I) (I on padding), X0 = I, split;
+// xscale = c^(1/4) with c = 1/(2 lambda).
+void launch_cn_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, __half* M0,
+                    __half* X0, float* xscale, cudaStream_t st);
+
 // Gather gradient blocks into padded split matrices: Gs[2k] = G_k, Gs[2k+1] = G_k^T.
 void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int B, __half* Gs, cudaStream_t st);
 

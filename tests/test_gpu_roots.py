@@ -164,3 +164,63 @@ def test_frobenius_scaling_roots(torch):
         assert abs(lam[i] - ref) <= 1e-5 * ref, (i, lam[i], ref)
     for i, r in enumerate(ndb_level2(A, 1e-6, lam, 20, 16)):
         assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
+
+
+def gpu_cn(torch, A, iters, fp16, eps=0.0, seed=0):
+    from matrix_inverse_roots_stack_b200 import binding as bd
+    B = A.shape[1]
+    v0 = torch.from_numpy(workloads.pi_start_vectors(B, 32, seed=seed)).cuda()
+    X, lam, ws = bd.inv_root_coupled_newton(torch.from_numpy(np.ascontiguousarray(A, dtype=np.float32)).cuda(),
+                                            v0, iters=iters, fp16=fp16, eps=eps)
+    rc, _ = bd.read_status(ws)
+    return X.cpu().numpy().astype(np.float64), lam.cpu().numpy().astype(np.float64), rc
+
+
+def cn_level2(A, eps, lam, iters):
+    return [roots.cn_inv4root_spectral(A[i].astype(np.float64) + eps * np.eye(A.shape[1]), lam[i], iters)
+            for i in range(A.shape[0])]
+
+
+@pytest.mark.parametrize("kappa,iters", [(1e2, 12), (1e3, 16), (1e4, 18)])
+def test_coupled_newton_split(torch, kappa, iters):
+    # split-fp16 products: within the root tolerance (measured 6e-7 .. 4e-5)
+    A = workloads.spd_stack_geometric(3, 256, kappa, seed=3)
+    X, lam, rc = gpu_cn(torch, A, iters, False)
+    assert rc == 0
+    for i, r in enumerate(cn_level2(A, 0.0, lam, iters)):
+        assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
+    # these counts converge: level 2 is the exact root here
+    for i in range(3):
+        assert rel(X[i], roots.inv_root_eigh(A[i].astype(np.float64))) < ROOT_TOL
+
+
+def test_coupled_newton_split_kappa_1e6(torch):
+    # the coupled iteration carries X without self-correction, so rounding in
+    # the early, far-from-converged steps stays: 2.7e-3 measured at kappa=1e6
+    # (Newton-DB: 0.8e-3); bound 5e-3
+    A = workloads.spd_stack_geometric(3, 128, 1e6, seed=3)
+    X, lam, rc = gpu_cn(torch, A, 24, False)
+    assert rc == 0
+    for i, r in enumerate(cn_level2(A, 0.0, lam, 24)):
+        assert rel(X[i], r) < 5e-3, (i, rel(X[i], r))
+
+
+@pytest.mark.parametrize("kappa,iters,tol", [(1e2, 12, 3e-3), (1e3, 16, 1.5e-2)])
+def test_coupled_newton_fp16(torch, kappa, iters, tol):
+    # single-pass fp16 operands (unit roundoff 2^-11 = 4.9e-4) with fp32
+    # accumulation: measured 1.0e-3 at kappa=1e2 and 5.7e-3 at 1e3 (bounds 3x)
+    A = workloads.spd_stack_geometric(3, 256, kappa, seed=3)
+    X, lam, rc = gpu_cn(torch, A, iters, True)
+    assert rc == 0
+    for i, r in enumerate(cn_level2(A, 0.0, lam, iters)):
+        assert rel(X[i], r) < tol, (i, rel(X[i], r))
+
+
+def test_coupled_newton_fp16_reports_divergence(torch):
+    # at kappa=1e6 fp16 rounding pushes small eigenvalues of M below zero and
+    # the iteration diverges; the status word says so instead of returning
+    # garbage silently
+    from matrix_inverse_roots_stack_b200 import binding as bd
+    A = workloads.spd_stack_geometric(3, 128, 1e6, seed=3)
+    X, lam, rc = gpu_cn(torch, A, 24, True)
+    assert rc == bd.SHAMPOO_ENONFINITE

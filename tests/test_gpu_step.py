@@ -29,7 +29,8 @@ def run_gpu(torch, thetas, grads, hp, steps=1, seed=0):
     from matrix_inverse_roots_stack_b200 import binding as bd
     h = bd.make_hparams(block_size=hp.block_size, beta=hp.beta, eps=hp.eps, init_scale=hp.init_scale,
                         beta1=hp.beta1, beta2=hp.beta2, adam_eps=hp.adam_eps, lr=hp.lr,
-                        solver=bd.SOLVER_NEWTON_DB if hp.solver == "ndb" else bd.SOLVER_CHEBYSHEV,
+                        solver={"ndb": bd.SOLVER_NEWTON_DB, "cheb": bd.SOLVER_CHEBYSHEV,
+                                "cn": bd.SOLVER_COUPLED_NEWTON}[hp.solver], cn_iters=hp.cn_iters,
                         ndb_iters1=hp.ndb_iters1, ndb_iters2=hp.ndb_iters2, cheb_degree=hp.cheb_degree,
                         cheb_delta=hp.cheb_delta, pi_iters=hp.pi_iters, root_every=hp.root_every,
                         scaling=bd.SCALING_FROBENIUS if hp.scaling == "frobenius" else bd.SCALING_SPECTRAL)
@@ -189,4 +190,13 @@ def test_frobenius_scaling_step(torch):
             ref = np.linalg.norm(Ab, "fro")
             assert abs(gpu["lam"][0][f] - ref) <= 1e-5 * ref, (f, gpu["lam"][0][f], ref)
             f += 1
+    compare(gpu, th, grads, hp)
+
+
+def test_coupled_newton_step(torch):
+    shapes = [(256, 384), (128, 200)]
+    grads = [[g] for g in workloads.gaussian_gradients(shapes, std=0.1, seed=24)]
+    th = workloads.parameters(shapes, seed=25)
+    hp = ostep.HParams(block_size=128, solver="cn", cn_iters=18, eps=1e-4)
+    gpu = run_gpu(torch, th, grads, hp)
     compare(gpu, th, grads, hp)

@@ -19,10 +19,12 @@ host cores on a bounded sample of the same workload.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload llama1b|gpt2|spiked512|roots256|mixed]
 
-For N > 1 (torchrun, one process per GPU) every rank runs its own replica of
-the workload (weak scaling; the blocks of different ranks are independent
-problems and no collective is on the data path); the step time is the max
-over ranks.
+For N > 1 (torchrun, one process per GPU) the parameters are shared out by
+greedy ownership (decreasing root cost, least-loaded rank first); each rank
+runs the step for the blocks of the parameters it owns and one NCCL
+all-gather per step gives every rank all updated parameters (strong scaling:
+the workload is fixed).  The step time is the max over ranks.  The standalone
+roots workload runs one replica per rank.
 """
 
 import argparse
@@ -313,16 +315,25 @@ def main():
                              cheb_degree=args.degree, root_every=args.root_every, cn_iters=args.cn_iters,
                              cn_fp16=1 if cn16 else 0,
                              scaling=bd.SCALING_FROBENIUS if args.scaling == "frobenius" else bd.SCALING_SPECTRAL)
-        opt = bd.Shampoo(params, grads, hp=hp,
-                         v0=torch.from_numpy(wl.pi_start_vectors(B, 32, seed=0)).to(dev))
-        bsz = block_sizes(spec["shapes"], B)
+        v0 = torch.from_numpy(wl.pi_start_vectors(B, 32, seed=0)).to(dev)
+        # one rank per GPU: greedy ownership of the parameters, each rank steps
+        # its own and one all-gather per step distributes the results
+        from matrix_inverse_roots_stack_b200 import distributed as sd
+        sharded = sd.ShardedShampoo(params, grads, B, make_local=lambda ps, gs: bd.Shampoo(ps, gs, hp=hp, v0=v0))
+        opt = sharded.local
+        if opt is None:
+            raise SystemExit(f"rank {rank} owns no parameter: use fewer GPUs for this workload")
+        owned_shapes = [tuple(params[i].shape) for i in sharded.owned]
+        bsz = block_sizes(owned_shapes, B)
         factor_sizes = [s for pair in bsz for s in pair]
         n_factors = opt.n_factors
-        ctx_info = {"n_params": len(params), "n_blocks": opt.n_blocks, "n_factors": opt.n_factors,
+        ctx_info = {"n_params": len(params), "n_blocks": len(block_sizes(spec["shapes"], B)),
+                    "n_factors": 2 * len(block_sizes(spec["shapes"], B)),
+                    "rank0_owned_params": len(sharded.owned), "rank0_n_factors": opt.n_factors,
                     "workspace_gb": round(opt.ws.numel() / 1e9, 2)}
 
         def step_fn():
-            opt.step()
+            sharded.step()
 
         def e2e_fn(host_g, host_p):
             # the same step through the C ABI with host buffers: upload the
@@ -332,7 +343,7 @@ def main():
                 n = g.numel()
                 g.view(-1).copy_(host_g[off:off + n], non_blocking=True)
                 off += n
-            opt.step()
+            sharded.step()
             off = 0
             for p in params:
                 n = p.numel()
@@ -457,7 +468,9 @@ def main():
 
     line = {"metric": "Shampoo optimizer step ms", "value": round(ms, 3), "unit": "ms", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (3 x fp16-split tensor products, fp32 accumulate)",
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": "f32 (3 x fp16-split tensor products, fp32 accumulate)" if args.solver != "cn16" else
+                     "f16 products, f32 accumulate",
             "data": "synthetic",
             "config": dict({"workload": spec["desc"], "block_size": B, "solver": args.solver,
                             "iters_per_stage": iters if args.solver == "ndb" else None,
@@ -467,7 +480,10 @@ def main():
                                                else "Frobenius norm"),
                             "roots_every_steps": max(1, args.root_every),
                             "l2": "working set far larger than the 126 MB L2 (no flush needed)",
-                            "parallelism": f"replicas x{world}"}, **ctx_info),
+                            "parallelism": ("one GPU" if world == 1 else
+                                            f"replicas x{world}" if spec["shapes"] is None else
+                                            f"sharded x{world}: greedy parameter ownership by root cost, "
+                                            "NCCL all-gather of the updated parameters")}, **ctx_info),
             "roofline": roofline, "inverse_root": inverse_root, "stage_ms": stages,
             "gpu_launches": prof["launches"], "clocks": clock_info, "e2e": e2e, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)

@@ -224,6 +224,29 @@ def oracle_sample(spec, args, budget_s=15.0, seed=0):
             f"{total_blocks} blocks, extrapolated x{frac:.1f} by block count", threads)
 
 
+def arm_config(args, spec, world):
+    """The workload description both arms report (identical dicts)."""
+    cfg = {"workload": spec["desc"], "block_size": spec["B"], "solver": args.solver,
+           "iters_per_stage": spec["iters"] if args.solver == "ndb" else None,
+           "cheb_degree": args.degree if args.solver == "cheb" else None,
+           "cn_iters": args.cn_iters if args.solver in ("cn", "cn16") else None,
+           "scale_estimate": ("power iteration, 10 products x 32 starts" if args.scaling == "spectral"
+                              else "Frobenius norm"),
+           "roots_every_steps": max(1, args.root_every),
+           "l2": ("working set far larger than the 126 MB L2 (no flush needed)" if spec["B"] >= 512 and
+                  spec["shapes"] is not None else "small working set, no L2 flush between steps (not a headline)"),
+           "parallelism": ("one GPU" if world == 1 else
+                           f"replicas x{world}" if spec["shapes"] is None else
+                           f"sharded x{world}: greedy parameter ownership by root cost, "
+                           "NCCL all-gather of the updated parameters")}
+    if spec["shapes"] is not None:
+        nb = len(block_sizes(spec["shapes"], spec["B"]))
+        cfg.update({"n_params": len(spec["shapes"]), "n_blocks": nb, "n_factors": 2 * nb})
+    else:
+        cfg["n_matrices"] = spec["n"]
+    return cfg
+
+
 def run_reference(args, spec, rank):
     if rank != 0:
         return
@@ -235,9 +258,8 @@ def run_reference(args, spec, rank):
     ms = statistics.median(per_step)
     line = {"impl": "reference", "metric": "Shampoo optimizer step ms", "value": round(ms, 3), "unit": "ms",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": spec["desc"], "block_size": spec["B"],
-                                            "solver": args.solver, "iters": spec["iters"]},
+            "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": arm_config(args, spec, args.gpus),
             "cpu_baseline": {"value": round(ms, 3), "unit": "ms", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -306,7 +328,7 @@ def main():
             else:
                 bd.inv_root_chebyshev(At, v0, args.degree, 1e-3, 0.0, 10, X, lam, ws)
         n_factors, factor_sizes = nmat, [B] * nmat
-        ctx_info = {"n_matrices": nmat}
+        ctx_info = {}
         e2e_fn = None
     else:
         grads = make_grads(spec, dev, seed=0)
@@ -327,9 +349,7 @@ def main():
         bsz = block_sizes(owned_shapes, B)
         factor_sizes = [s for pair in bsz for s in pair]
         n_factors = opt.n_factors
-        ctx_info = {"n_params": len(params), "n_blocks": len(block_sizes(spec["shapes"], B)),
-                    "n_factors": 2 * len(block_sizes(spec["shapes"], B)),
-                    "rank0_owned_params": len(sharded.owned), "rank0_n_factors": opt.n_factors,
+        ctx_info = {"rank0_owned_params": len(sharded.owned), "rank0_n_factors": opt.n_factors,
                     "workspace_gb": round(opt.ws.numel() / 1e9, 2)}
 
         def step_fn():
@@ -472,18 +492,7 @@ def main():
             "dtype": "f32 (3 x fp16-split tensor products, fp32 accumulate)" if args.solver != "cn16" else
                      "f16 products, f32 accumulate",
             "data": "synthetic",
-            "config": dict({"workload": spec["desc"], "block_size": B, "solver": args.solver,
-                            "iters_per_stage": iters if args.solver == "ndb" else None,
-                            "cheb_degree": args.degree if args.solver == "cheb" else None,
-                            "cn_iters": args.cn_iters if args.solver in ("cn", "cn16") else None,
-                            "scale_estimate": ("power iteration, 10 products x 32 starts" if args.scaling == "spectral"
-                                               else "Frobenius norm"),
-                            "roots_every_steps": max(1, args.root_every),
-                            "l2": "working set far larger than the 126 MB L2 (no flush needed)",
-                            "parallelism": ("one GPU" if world == 1 else
-                                            f"replicas x{world}" if spec["shapes"] is None else
-                                            f"sharded x{world}: greedy parameter ownership by root cost, "
-                                            "NCCL all-gather of the updated parameters")}, **ctx_info),
+            "config": arm_config(args, spec, world), "state": ctx_info,
             "roofline": roofline, "inverse_root": inverse_root, "stage_ms": stages,
             "gpu_launches": prof["launches"], "clocks": clock_info, "e2e": e2e, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)

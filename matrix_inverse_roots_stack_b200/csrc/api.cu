@@ -558,7 +558,7 @@ int shampoo_init_blocks(shampoo_ctx** out, const shampoo_param* params, int n_pa
     c->pdev.push_back(d);
     c->prefix.push_back(items);
     uoff += q.rows * q.cols;
-    items += q.rows * static_cast<long long>(d.chunks);
+    items += ((q.rows + dash::kUpdRows - 1) / dash::kUpdRows) * static_cast<long long>(d.chunks);
   }
   c->prefix.push_back(items);
   c->n_items = items;

@@ -403,8 +403,11 @@ __global__ void init_factors_kernel(float* __restrict__ F, int B, float s) {
 //
 // DASH explainer, "Step-by-step" (grafting with Adam's magnitude): P is the
 // Adam direction, s = ||P||_F / ||U||_F per block, theta -= lr * s * U.
-// One CTA = one work item = up to 1024 columns of one row of one parameter;
-// a warp covers 128 aligned columns, which lie in one block (B % 128 == 0).
+// One CTA = one work item = kUpdRows rows x up to 1024 columns of one
+// parameter; a warp covers 128 aligned columns, which lie in one block
+// (B % 128 == 0), and the rows of an item lie in one block row (B % 8 == 0),
+// so each warp's sum of P^2 belongs to one block.  Warps of the same block
+// are combined in shared memory before the one atomic per block and item.
 
 __device__ __forceinline__ int find_param(const long long* prefix, int n, long long item) {
   int lo = 0, hi = n - 1;
@@ -416,58 +419,80 @@ __device__ __forceinline__ int find_param(const long long* prefix, int n, long l
   return lo;
 }
 
+__device__ __forceinline__ void adam4(const float* g, float* m, float* v, float b1, float b2, float eps, float ibc1,
+                                      float ibc2, float& sq) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    m[e] = b1 * m[e] + (1.0f - b1) * g[e];
+    v[e] = b2 * v[e] + (1.0f - b2) * g[e] * g[e];
+    const float p = (m[e] * ibc1) / (sqrtf(v[e] * ibc2) + eps);
+    sq += p * p;
+  }
+}
+
 __global__ void __launch_bounds__(256) adam_kernel(const ParamDev* __restrict__ params,
                                                    const long long* __restrict__ prefix, int n_params, int B,
                                                    float b1, float b2, float eps, float ibc1, float ibc2,
                                                    float* __restrict__ pnorm) {
+  __shared__ float wsum[8];
+  __shared__ int wblk[8];
   const long long item = blockIdx.x;
   const int pi = find_param(prefix, n_params, item);
   const ParamDev P = params[pi];
   const long long local = item - P.item_base;
-  const int r = static_cast<int>(local / P.chunks);
+  const int r0 = static_cast<int>(local / P.chunks) * kUpdRows;
   const int c0 = static_cast<int>(local % P.chunks) * 1024;
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = c0 + threadIdx.x * 4;
-  const size_t base = static_cast<size_t>(r) * P.cols;
+  const int r1 = min(r0 + kUpdRows, P.rows);
   float sq = 0.0f;
-  if (P.vec) {
-    if (c < P.cols) {
-      const float4 g = *reinterpret_cast<const float4*>(P.grad + base + c);
-      float4 m = *reinterpret_cast<const float4*>(P.m + base + c);
-      float4 v = *reinterpret_cast<const float4*>(P.v + base + c);
-      const float gv[4] = {g.x, g.y, g.z, g.w};
-      float mv[4] = {m.x, m.y, m.z, m.w}, vv[4] = {v.x, v.y, v.z, v.w};
+  for (int r = r0; r < r1; ++r) {
+    const size_t base = static_cast<size_t>(r) * P.cols;
+    if (P.vec) {
+      if (c < P.cols) {
+        const float4 g4 = *reinterpret_cast<const float4*>(P.grad + base + c);
+        const float4 m4 = *reinterpret_cast<const float4*>(P.m + base + c);
+        const float4 v4 = *reinterpret_cast<const float4*>(P.v + base + c);
+        const float g[4] = {g4.x, g4.y, g4.z, g4.w};
+        float m[4] = {m4.x, m4.y, m4.z, m4.w}, v[4] = {v4.x, v4.y, v4.z, v4.w};
+        adam4(g, m, v, b1, b2, eps, ibc1, ibc2, sq);
+        *reinterpret_cast<float4*>(P.m + base + c) = make_float4(m[0], m[1], m[2], m[3]);
+        *reinterpret_cast<float4*>(P.v + base + c) = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        mv[e] = b1 * mv[e] + (1.0f - b1) * gv[e];
-        vv[e] = b2 * vv[e] + (1.0f - b2) * gv[e] * gv[e];
-        const float p = (mv[e] * ibc1) / (sqrtf(vv[e] * ibc2) + eps);
-        sq += p * p;
-      }
-      *reinterpret_cast<float4*>(P.m + base + c) = make_float4(mv[0], mv[1], mv[2], mv[3]);
-      *reinterpret_cast<float4*>(P.v + base + c) = make_float4(vv[0], vv[1], vv[2], vv[3]);
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int ce = c + e;
-      if (ce < P.cols) {
-        const float g = P.grad[base + ce];
-        const float m = b1 * P.m[base + ce] + (1.0f - b1) * g;
-        const float v = b2 * P.v[base + ce] + (1.0f - b2) * g * g;
-        P.m[base + ce] = m;
-        P.v[base + ce] = v;
-        const float p = (m * ibc1) / (sqrtf(v * ibc2) + eps);
-        sq += p * p;
+        const int ce = c + e;
+        if (ce < P.cols) {
+          const float g = P.grad[base + ce];
+          const float m = b1 * P.m[base + ce] + (1.0f - b1) * g;
+          const float v = b2 * P.v[base + ce] + (1.0f - b2) * g * g;
+          P.m[base + ce] = m;
+          P.v[base + ce] = v;
+          const float p = (m * ibc1) / (sqrtf(v * ibc2) + eps);
+          sq += p * p;
+        }
       }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   const int cw = c0 + warp * 128;
-  if ((threadIdx.x & 31) == 0 && cw < P.cols && sq != 0.0f) {
-    const int k = P.blk_base + (r / B) * P.ncb + cw / B;
-    atomicAdd(&pnorm[k], sq);
+  if (lane == 0) {
+    wsum[warp] = sq;
+    wblk[warp] = cw < P.cols ? P.blk_base + (r0 / B) * P.ncb + cw / B : -1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // one atomic per block the item touches
+    float acc = 0.0f;
+    for (int w = 0; w < 8; ++w) {
+      if (wblk[w] < 0) break;
+      acc += wsum[w];
+      if (w == 7 || wblk[w + 1] != wblk[w]) {
+        if (acc != 0.0f) atomicAdd(&pnorm[wblk[w]], acc);
+        acc = 0.0f;
+      }
+    }
   }
 }
 
@@ -480,27 +505,30 @@ __global__ void __launch_bounds__(256) update_kernel(const ParamDev* __restrict_
   const int pi = find_param(prefix, n_params, item);
   const ParamDev P = params[pi];
   const long long local = item - P.item_base;
-  const int r = static_cast<int>(local / P.chunks);
+  const int r0 = static_cast<int>(local / P.chunks) * kUpdRows;
   const int c0 = static_cast<int>(local % P.chunks) * 1024;
   const int c = c0 + threadIdx.x * 4;
   if (c >= P.cols) return;
-  const int k = P.blk_base + (r / B) * P.ncb + c / B;
+  const int k = P.blk_base + (r0 / B) * P.ncb + c / B;
   const float un = unorm[k];
   const float s = un > 0.0f ? lr * sqrtf(pnorm[k] / un) : 0.0f;
-  const size_t base = static_cast<size_t>(r) * P.cols;
-  const float* u = U + P.uoff + base;
-  if (P.vec) {
-    float4 th = *reinterpret_cast<const float4*>(P.param + base + c);
-    const float4 uu = *reinterpret_cast<const float4*>(u + c);
-    th.x -= s * uu.x;
-    th.y -= s * uu.y;
-    th.z -= s * uu.z;
-    th.w -= s * uu.w;
-    *reinterpret_cast<float4*>(P.param + base + c) = th;
-  } else {
+  const int r1 = min(r0 + kUpdRows, P.rows);
+  for (int r = r0; r < r1; ++r) {
+    const size_t base = static_cast<size_t>(r) * P.cols;
+    const float* u = U + P.uoff + base;
+    if (P.vec) {
+      float4 th = *reinterpret_cast<const float4*>(P.param + base + c);
+      const float4 uu = *reinterpret_cast<const float4*>(u + c);
+      th.x -= s * uu.x;
+      th.y -= s * uu.y;
+      th.z -= s * uu.z;
+      th.w -= s * uu.w;
+      *reinterpret_cast<float4*>(P.param + base + c) = th;
+    } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if (c + e < P.cols) P.param[base + c + e] -= s * u[c + e];
+      for (int e = 0; e < 4; ++e)
+        if (c + e < P.cols) P.param[base + c + e] -= s * u[c + e];
+    }
   }
 }
 

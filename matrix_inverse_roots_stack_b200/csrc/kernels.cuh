@@ -13,13 +13,17 @@ namespace dash {
 constexpr int kPiStarts = 32;  // power-iteration start vectors per factor
 
 // Per-parameter metadata used by the Adam / update kernels.
+// Rows per Adam / update work item (one item = kUpdRows rows x up to 1024
+// columns of one parameter).
+constexpr int kUpdRows = 8;
+
 struct ParamDev {
   const float* grad;
   float* param;
   float* m;
   float* v;
   long long uoff;       // offset of this parameter in the flat U buffer
-  long long item_base;  // first work item (one item = 1024 columns of one row)
+  long long item_base;  // first work item (kUpdRows rows x 1024 columns)
   int rows, cols;
   int blk_base;         // index of the parameter's first block
   int ncb;              // column blocks

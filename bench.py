@@ -40,6 +40,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+
+# DRAM bytes (read + write) per executed tensor-core flop of gemm_split_kernel,
+# by (block size, solver): from an ncu capture of every GEMM launch of one step
+# of the mixed-shape B=1024 workload (profiles/gemm_split_kernel_traffic_b1024_ndb14.md).
+# Each launch reads and writes its problems' split matrices about once, so a
+# launch's traffic grows in proportion to the problems, and executed flops, it
+# covers; the roofline's per-launch traffic scales this ratio by those flops.
+GEMM_DRAM_BYTES_PER_FLOP = {(1024, "ndb"): 1.606e-3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -448,10 +456,13 @@ def main():
     avg_ms = g_ms / max(g_n, 1)
     # executed fp16 MMA flops as the library records them (3 per useful product, 1 in fp16 mode)
     achieved = (g_flops / max(g_n, 1)) / (avg_ms * 1e-3) / 1e12 if g_n else None
+    bpf = GEMM_DRAM_BYTES_PER_FLOP.get((B, args.solver))
+    traffic = round(bpf * g_flops / g_n) if (bpf and g_n) else None
     roofline = {"kernel": "gemm_split_kernel", "bound": "tensor",
                 "achieved": round(achieved, 1) if achieved else None, "peak": tensor_peak,
                 "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4) if achieved else None,
-                "traffic": None, "peak_kind": f"{peak_kind} bf16/fp16 dense, sustained",
+                "traffic": traffic, "traffic_unit": "bytes per launch (ncu DRAM read+write, scaled by executed flops)"
+                if traffic else None, "peak_kind": f"{peak_kind} bf16/fp16 dense, sustained",
                 "launches": g_n, "avg_launch_ms": round(avg_ms, 4),
                 "share_of_step": round(g_ms / (ms * args.steps), 4)}
 

@@ -52,7 +52,7 @@ int solver_chunk(int nf, int B, int solver) {
 
 // Workspace of the root solvers for nf factors of size B.
 struct RootLayout {
-  size_t status, lam, xscale, stats, w0, w1, solver;
+  size_t status, lam, xscale, pscale, stats, w0, w1, vt, solver;
   int chunk;
 };
 
@@ -63,9 +63,13 @@ void plan_roots(Bump& b, RootLayout& L, int nf, int B, int pi_iters, int extra_m
   L.stats = b.take(sizeof(float) * static_cast<size_t>(pi_iters) * nf * 3 * dash::kPiStarts);
   L.w0 = b.take(sizeof(float) * static_cast<size_t>(nf) * B * dash::kPiStarts);
   L.w1 = b.take(sizeof(float) * static_cast<size_t>(nf) * B * dash::kPiStarts);
+  L.pscale = b.take(sizeof(float) * nf);
+  L.vt = b.take(2 * sizeof(__half) * static_cast<size_t>(nf) * B * dash::kPiStarts);
   L.chunk = solver_chunk(nf, B, solver);
   const int per = solver_mats(solver);
-  const int mats = per * L.chunk > extra_mats ? per * L.chunk : extra_mats;
+  // the solver scratch also holds the split factors during the power iteration
+  int mats = per * L.chunk > extra_mats ? per * L.chunk : extra_mats;
+  if (mats < nf) mats = nf;
   L.solver = b.take(split_bytes(mats, B));
 }
 
@@ -399,13 +403,21 @@ int run_roots(const float* F, int nf, int B, float eps, const int* fsize, const 
     dash::launch_frob_norm(F, nf, B, eps, fsize, lam, lam_out, st);
     DASH_LAUNCHED();
   } else {  // multi-start power iteration ("Building blocks", Multi-Power-Iteration)
+    // the split factors live in the solver scratch until the solver starts
+    __half* As = reinterpret_cast<__half*>(ws + L.solver);
+    __half* Vt = reinterpret_cast<__half*>(ws + L.vt);
+    float* pscale = reinterpret_cast<float*>(ws + L.pscale);
     DASH_TRY(cudaMemsetAsync(stats, 0, sizeof(float) * sstride * pi_iters, st));
+    dash::launch_pi_prepare(F, nf, B, eps, fsize, pscale, As, status, st);
+    DASH_LAUNCHED();
     for (int t = 0; t < pi_iters; ++t) {
-      dash::launch_pi_iter(F, nf, B, eps, fsize, v0, t ? W[(t - 1) & 1] : nullptr,
-                           t ? stats + (t - 1) * sstride : nullptr, W[t & 1], stats + t * sstride, st);
+      const float* Wp = t ? W[(t - 1) & 1] : nullptr;
+      const float* sp = t ? stats + (t - 1) * sstride : nullptr;
+      dash::launch_pi_vectors(v0, Wp, sp, nf, B, fsize, Vt, st);
       DASH_LAUNCHED();
+      DASH_TRY(dash::launch_pi_product(As, Vt, v0, Wp, sp, nf, B, fsize, W[t & 1], stats + t * sstride, status, st));
     }
-    dash::launch_pi_finalize(stats + (pi_iters - 1) * sstride, nf, lam, lam_out, st);
+    dash::launch_pi_finalize(stats + (pi_iters - 1) * sstride, nf, pscale, lam, lam_out, st);
     DASH_LAUNCHED();
   }
   dash::prof_end(pslot, st);

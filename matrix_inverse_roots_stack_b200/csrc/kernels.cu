@@ -6,179 +6,6 @@
 namespace dash {
 namespace {
 
-// ------------------------------------------------------------ power iteration
-//
-// DASH explainer, "Building blocks" (Multi-Power-Iteration): K random starts,
-// repeated products with the factor, largest Rayleigh quotient.  One CTA
-// computes 128 rows of W = A V (32 columns) for one factor, streaming A in
-// 128 x 32 slabs through shared memory.
-
-constexpr int kPiRows = 128;  // rows of W per CTA
-constexpr int kPiK = 32;      // K chunk per shared-memory stage
-constexpr int kPiPad = 4;     // padding of the transposed A tile (bank spread)
-
-// One chunk of the factor (128 rows x 32 k) and of V (32 k x 32 starts),
-// held in registers between global loads and shared-memory stores.
-struct PiChunk {
-  float4 a[4];
-  float4 v;
-};
-
-__device__ __forceinline__ PiChunk pi_load(const float* __restrict__ Fm, const float* __restrict__ Vsrc,
-                                           const float* inv, int B, int b, int r0, int k0, float eps, int t) {
-  PiChunk c;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {  // 1024 float4 of A: row = f / 8, k quad = f % 8
-    const int f = t + 256 * j;
-    const int rr = r0 + f / 8, kk = k0 + 4 * (f % 8);
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (rr < b) {
-      if (kk + 3 < b) {
-        x = *reinterpret_cast<const float4*>(Fm + static_cast<size_t>(rr) * B + kk);
-      } else {
-        float tmp[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) tmp[e] = (kk + e < b) ? Fm[static_cast<size_t>(rr) * B + kk + e] : 0.0f;
-        x = make_float4(tmp[0], tmp[1], tmp[2], tmp[3]);
-      }
-      if (rr >= kk && rr < kk + 4) {  // regulariser on the diagonal
-        if (rr == kk) x.x += eps;
-        if (rr == kk + 1) x.y += eps;
-        if (rr == kk + 2) x.z += eps;
-        if (rr == kk + 3) x.w += eps;
-      }
-    }
-    c.a[j] = x;
-  }
-  {  // 256 float4 of V: k = t / 8, columns 4 * (t % 8)
-    const int kk = k0 + t / 8, cc = 4 * (t % 8);
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (kk < b) {
-      x = *reinterpret_cast<const float4*>(Vsrc + static_cast<size_t>(kk) * kPiStarts + cc);
-      x.x *= inv[cc];
-      x.y *= inv[cc + 1];
-      x.z *= inv[cc + 2];
-      x.w *= inv[cc + 3];
-    }
-    c.v = x;
-  }
-  return c;
-}
-
-__device__ __forceinline__ void pi_store(const PiChunk& c, float (*As)[kPiRows + kPiPad], float (*Vs)[kPiStarts],
-                                         int t) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int f = t + 256 * j;
-    const int rr = f / 8, kq = 4 * (f % 8);
-    As[kq][rr] = c.a[j].x;
-    As[kq + 1][rr] = c.a[j].y;
-    As[kq + 2][rr] = c.a[j].z;
-    As[kq + 3][rr] = c.a[j].w;
-  }
-  *reinterpret_cast<float4*>(&Vs[t / 8][4 * (t % 8)]) = c.v;
-}
-
-__global__ void __launch_bounds__(256) pi_iter_kernel(const float* __restrict__ F, int B, float eps,
-                                                      const int* __restrict__ fsize, const float* __restrict__ v0,
-                                                      const float* __restrict__ Wprev,
-                                                      const float* __restrict__ sprev, float* __restrict__ Wnext,
-                                                      float* __restrict__ snext) {
-  __shared__ __align__(16) float As[kPiK][kPiRows + kPiPad];  // transposed: As[k][row]
-  __shared__ __align__(16) float Vs[kPiK][kPiStarts];
-  __shared__ float inv[kPiStarts];
-  __shared__ float red[3][32][kPiStarts + 1];
-
-  const int f = blockIdx.y;
-  const int r0 = blockIdx.x * kPiRows;
-  const int b = fsize ? fsize[f] : B;
-  const int t = threadIdx.x;
-  const int ty = t >> 3, tx = t & 7;  // rows 4ty..4ty+3, columns 4tx..4tx+3
-  if (t < kPiStarts) {
-    const float n2 = Wprev ? sprev[static_cast<size_t>(f) * 3 * kPiStarts + t] : 1.0f;
-    inv[t] = Wprev ? (n2 > 0.0f ? rsqrtf(n2) : 0.0f) : 1.0f;
-  }
-  __syncthreads();
-
-  const float* Fm = F + static_cast<size_t>(f) * B * B;
-  const float* Vsrc = Wprev ? Wprev + static_cast<size_t>(f) * B * kPiStarts : v0;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-
-  if (r0 < b) {
-    PiChunk nxt = pi_load(Fm, Vsrc, inv, B, b, r0, 0, eps, t);
-    for (int k0 = 0; k0 < b; k0 += kPiK) {
-      __syncthreads();
-      pi_store(nxt, As, Vs, t);
-      __syncthreads();
-      if (k0 + kPiK < b) nxt = pi_load(Fm, Vsrc, inv, B, b, r0, k0 + kPiK, eps, t);
-#pragma unroll 8
-      for (int kk = 0; kk < kPiK; ++kk) {
-        const float4 a = *reinterpret_cast<const float4*>(&As[kk][4 * ty]);
-        const float4 v = *reinterpret_cast<const float4*>(&Vs[kk][4 * tx]);
-        const float av[4] = {a.x, a.y, a.z, a.w};
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] += av[i] * vv[j];
-      }
-    }
-  }
-
-  // write W rows and accumulate the column statistics of this CTA's rows
-  float w2[4] = {0.f, 0.f, 0.f, 0.f}, vw[4] = {0.f, 0.f, 0.f, 0.f}, v2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int gr = r0 + 4 * ty + i;
-    float* Wo = Wnext + static_cast<size_t>(f) * B * kPiStarts + static_cast<size_t>(gr) * kPiStarts + 4 * tx;
-    *reinterpret_cast<float4*>(Wo) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-    float4 vr = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (gr < b) vr = *reinterpret_cast<const float4*>(Vsrc + static_cast<size_t>(gr) * kPiStarts + 4 * tx);
-    const float vv[4] = {vr.x * inv[4 * tx], vr.y * inv[4 * tx + 1], vr.z * inv[4 * tx + 2], vr.w * inv[4 * tx + 3]};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      w2[j] += acc[i][j] * acc[i][j];
-      vw[j] += vv[j] * acc[i][j];
-      v2[j] += vv[j] * vv[j];
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    red[0][ty][4 * tx + j] = w2[j];
-    red[1][ty][4 * tx + j] = vw[j];
-    red[2][ty][4 * tx + j] = v2[j];
-  }
-  __syncthreads();
-  if (t < 3 * kPiStarts) {
-    const int q = t / kPiStarts, c = t % kPiStarts;
-    float s = 0.0f;
-#pragma unroll 8
-    for (int y = 0; y < 32; ++y) s += red[q][y][c];
-    if (s != 0.0f) atomicAdd(&snext[static_cast<size_t>(f) * 3 * kPiStarts + q * kPiStarts + c], s);
-  }
-}
-
-__global__ void pi_finalize_kernel(const float* __restrict__ s, int nf, float* __restrict__ lam,
-                                   float* __restrict__ lam_out) {
-  const int f = blockIdx.x * blockDim.x + threadIdx.x;
-  if (f >= nf) return;
-  const float* sf = s + static_cast<size_t>(f) * 3 * kPiStarts;
-  float best = 0.0f;
-  bool any = false;
-  for (int j = 0; j < kPiStarts; ++j) {
-    const float den = sf[2 * kPiStarts + j];
-    const float rq = den > 0.0f ? sf[kPiStarts + j] / den : 0.0f;
-    if (!any || rq > best) best = rq;
-    any = true;
-  }
-  lam[f] = best;
-  if (lam_out) lam_out[f] = best;
-}
-
 // Frobenius-norm scale estimate ("Building blocks", scaling: the Frobenius
 // alternative to spectral scaling): lambda_f = ||F_f + eps I||_F over the
 // factor's real b x b part (padding excluded).  One CTA per factor, float64
@@ -535,19 +362,6 @@ __global__ void __launch_bounds__(256) update_kernel(const ParamDev* __restrict_
 }  // namespace
 
 // ------------------------------------------------------------ launchers
-
-void launch_pi_iter(const float* F, int nf, int B, float eps, const int* fsize, const float* v0,
-                    const float* W_prev, const float* stats_prev, float* W_next, float* stats_next,
-                    cudaStream_t st) {
-  dim3 grid(B / kPiRows, nf);
-  pi_iter_kernel<<<grid, 256, 0, st>>>(F, B, eps, fsize, v0, W_prev, stats_prev, W_next, stats_next);
-  prof_count_launch();
-}
-
-void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* lambda_out, cudaStream_t st) {
-  pi_finalize_kernel<<<(nf + 127) / 128, 128, 0, st>>>(stats_last, nf, lambda, lambda_out);
-  prof_count_launch();
-}
 
 void launch_frob_norm(const float* F, int nf, int B, float eps, const int* fsize, float* lambda, float* lambda_out,
                       cudaStream_t st) {

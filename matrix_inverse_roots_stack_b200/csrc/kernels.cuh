@@ -31,16 +31,31 @@ struct ParamDev {
   int vec;              // 1: float4 path (cols % 4 == 0, 16-byte aligned)
 };
 
-// Power iteration: one product W_next = (F + eps I) V on every factor, where
-// V = v0 (first product, t = 0) or W_prev with unit columns.  Rows/columns at
-// or beyond a factor's true size are treated as zero.  Accumulates per column
-// ||W_next||^2, V.W_next and V.V into stats_next ((nf, 3, 32), zeroed).
-void launch_pi_iter(const float* F, int nf, int B, float eps, const int* fsize, const float* v0,
-                    const float* W_prev, const float* stats_prev, float* W_next, float* stats_next,
-                    cudaStream_t st);
+// Power iteration on the tensor cores (power.cu).
+// pi_prepare: pscale[f] = 2^-e with 2^(e-1) <= max_i (F_ii + eps) < 2^e, and
+// As (a split stack of nf matrices) = (F + eps I) pscale on each factor's
+// real part, 0 on the padding.
+void launch_pi_prepare(const float* F, int nf, int B, float eps, const int* fsize, float* pscale, __half* As,
+                       unsigned* status, cudaStream_t st);
 
-// lambda[f] = max_j (V.W)_j / (V.V)_j from the last product's statistics.
-void launch_pi_finalize(const float* stats_last, int nf, float* lambda, float* lambda_out, cudaStream_t st);
+// pi_vectors: Vt ((nf, 2, 32, B) fp16, hi/lo planes) = the next product's
+// input vectors, transposed: v0 ((B, 32) fp32, shared by all factors) when
+// W_prev is null, else W_prev ((nf, B, 32) fp32) with unit columns (norms
+// from stats_prev).  Rows at or beyond a factor's true size are 0.
+void launch_pi_vectors(const float* v0, const float* W_prev, const float* stats_prev, int nf, int B,
+                       const int* fsize, __half* Vt, cudaStream_t st);
+
+// pi_product: W_next = As V (V the split operand of pi_vectors; W_next is
+// scaled by pscale like As) and, per column, |W_next|^2, V.W_next and V.V
+// accumulated into stats_next ((nf, 3, 32), zeroed beforehand).
+cudaError_t launch_pi_product(const __half* As, const __half* Vt, const float* v0, const float* W_prev,
+                              const float* stats_prev, int nf, int B, const int* fsize, float* W_next,
+                              float* stats_next, unsigned* status, cudaStream_t st);
+
+// lambda[f] = max_j (V.W)_j / (V.V)_j / pscale[f] from the last product's
+// statistics (pscale may be null: 1).
+void launch_pi_finalize(const float* stats_last, int nf, const float* pscale, float* lambda, float* lambda_out,
+                        cudaStream_t st);
 
 // lambda_f = ||F_f + eps I||_F over the real fsize[f] x fsize[f] part (the
 // Frobenius scale estimate, in place of the power iteration).

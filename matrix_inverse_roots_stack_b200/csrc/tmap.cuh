@@ -9,6 +9,12 @@
 
 namespace dash {
 
+// Encode a 3-D tiled map over fp16 data laid out as depth x rows x cols
+// (cols innermost, cols a multiple of 64): box {64, box_rows, 1}, 128-byte
+// swizzle.  Returns cudaSuccess or cudaErrorInvalidValue.
+cudaError_t encode_f16_3d_map(CUtensorMap* map, const void* base, int cols, int rows, long long depth,
+                              int box_rows);
+
 // Encode a 3-D tiled map over a split stack: dims {B (columns, innermost),
 // B (rows), 2 * nmat (matrix * 2 + plane)} of fp16, box {64, box_rows, 1},
 // 128-byte swizzle.  Returns cudaSuccess or cudaErrorInvalidValue.

@@ -70,6 +70,9 @@ def parse_args():
                    help="recompute roots every F-th step and reuse them in between (default: every step)")
     p.add_argument("--scaling", default="spectral", choices=["spectral", "frobenius"])
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--e2e-groups", type=int, default=4,
+                   help="parameter groups of the host-buffer step on one GPU (copies overlap the other "
+                        "groups' work); 1: upload, step and download one after the other")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -350,6 +353,7 @@ def main():
         # its own and one all-gather per step distributes the results
         from matrix_inverse_roots_stack_b200 import distributed as sd
         sharded = sd.ShardedShampoo(params, grads, B, make_local=lambda ps, gs: bd.Shampoo(ps, gs, hp=hp, v0=v0))
+        live = {"sharded": sharded}
         opt = sharded.local
         if opt is None:
             raise SystemExit(f"rank {rank} owns no parameter: use fewer GPUs for this workload")
@@ -361,17 +365,20 @@ def main():
                     "workspace_gb": round(opt.ws.numel() / 1e9, 2)}
 
         def step_fn():
-            sharded.step()
+            live["sharded"].step()
 
         def e2e_fn(host_g, host_p):
             # the same step through the C ABI with host buffers: upload the
             # step's gradients from pinned memory, step, read the parameters back
+            if "pipe" in live:  # one GPU: copies overlapped with the other groups' work
+                live["pipe"].step(live["hg"], live["hp"])
+                return
             off = 0
             for g in grads:
                 n = g.numel()
                 g.view(-1).copy_(host_g[off:off + n], non_blocking=True)
                 off += n
-            sharded.step()
+            live["sharded"].step()
             off = 0
             for p in params:
                 n = p.numel()
@@ -423,6 +430,28 @@ def main():
             for g in grads:
                 host_g[off:off + g.numel()].copy_(g.view(-1).cpu())
                 off += g.numel()
+            if world == 1 and args.e2e_groups > 1:
+                # the pipelined host-buffer step keeps its own device state: release
+                # the device-resident optimizer first
+                from matrix_inverse_roots_stack_b200.pipeline import HostPipelinedShampoo
+                live.clear()
+                opt = sharded = None
+                torch.cuda.empty_cache()
+                pipe = HostPipelinedShampoo([tuple(p.shape) for p in params], hp=hp, v0=v0, device=dev,
+                                            groups=args.e2e_groups)
+                hg, hpl, off = [], [], 0
+                for p in params:
+                    n = p.numel()
+                    hg.append(host_g[off:off + n].view(p.shape))
+                    hpl.append(host_p[off:off + n].view(p.shape))
+                    host_p[off:off + n].copy_(p.view(-1).cpu())
+                    off += n
+                pipe.load_params(hpl)
+                live.update(pipe=pipe, hg=hg, hp=hpl)
+                e2e_info = {"groups": len(pipe.groups), "overlap": "uploads, steps and downloads of groups "
+                            "on three streams"}
+            else:
+                e2e_info = {"groups": 1, "overlap": "none"}
             e2e_fn(host_g, host_p)
             torch.cuda.synchronize()
             barrier()
@@ -439,7 +468,7 @@ def main():
                 dist.all_reduce(t, op=dist.ReduceOp.MAX)
                 e_ms = float(t.item())
             e2e = {"value": round(e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 4 * n_g,
-                   "d2h_bytes_per_step": 4 * n_p}
+                   "d2h_bytes_per_step": 4 * n_p, **e2e_info}
             del host_g, host_p
         except RuntimeError as exc:
             e2e = {"value": None, "unit": "ms", "error": str(exc)[:200]}

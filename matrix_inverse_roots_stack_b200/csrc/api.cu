@@ -538,6 +538,9 @@ int shampoo_init_blocks(shampoo_ctx** out, const shampoo_param* params, int n_pa
   long long uoff = 0, items = 0;
   for (int p = 0; p < n_params; ++p) {
     const shampoo_param& q = params[p];
+    // each parameter's slice of the flat U buffer starts on 16 bytes, so the
+    // float4 path of the update reads it aligned whatever the sizes before it
+    uoff = (uoff + 3) & ~3ll;
     ParamDev d;
     d.grad = q.grad;
     d.param = q.param;

@@ -126,7 +126,9 @@ def test_spiked_512_single_weight(torch):
 
 
 def test_ragged_edges_multi_param(torch):
-    shapes = [(300, 200), (128, 520), (5, 7)]
+    # (5, 7) has 35 elements, so the (64, 132) parameter after it exercises
+    # the 16-byte alignment of its slice of the flat U buffer (float4 path)
+    shapes = [(300, 200), (128, 520), (5, 7), (64, 132)]
     grads = [[g] for g in workloads.gaussian_gradients(shapes, std=0.1, seed=3)]
     th = workloads.parameters(shapes, seed=4)
     hp = ostep.HParams(block_size=128, ndb_iters1=12, ndb_iters2=12)
@@ -135,6 +137,7 @@ def test_ragged_edges_multi_param(torch):
     expect = [(p, r0, c0, r1 - r0, c1 - c0) for p, s in enumerate(shapes)
               for (r0, r1, c0, c1) in ostep.block_grid(*s, 128)]
     assert [tuple(r[:5]) for r in tab] == expect
+    check_lambdas(gpu, grads, hp)  # factors of 44, 8, 5, 7, 64 and 4 inside 128-padded storage
     compare(gpu, th, grads, hp)
 
 

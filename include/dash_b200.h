@@ -28,7 +28,12 @@
  *    read it with shampoo_read_status after the call.
  *  - Power iteration uses caller-supplied start vectors `v0` (device, fp32,
  *    B x 32 row-major: column j is start vector j).  A factor of true size
- *    b < B uses rows 0..b-1.
+ *    b < B uses rows 0..b-1.  Its products run on the tensor cores with
+ *    split-fp16 operands: each A + eps I is first scaled by the power of two
+ *    2^-e with 2^(e-1) <= its largest diagonal entry < 2^e, which keeps every
+ *    entry of a positive semi-definite matrix within [-1, 1] (exact scaling;
+ *    lambda is returned unscaled).  A matrix with an entry beyond 65504 * 2^e
+ *    (not positive semi-definite) sets the status word's non-finite bit.
  *  - Return value: 0 on success or a negative SHAMPOO_E* code.  No C++
  *    exception crosses this boundary.  On an error return nothing has been
  *    enqueued unless the code is SHAMPOO_ECUDA.

@@ -170,14 +170,29 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
+        note = None
+        if not rows:
+            # the timed region ended before the sampler's first reading: take
+            # one reading now, right after it
+            try:
+                q = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+                rows = [[x.strip() for x in line.split(",")] for line in q.stdout.splitlines()
+                        if len(line.split(",")) >= 9]
+                note = "timed region shorter than the sampler's start-up: one reading right after it"
+            except (OSError, subprocess.SubprocessError):
+                rows = []
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+               "reasons": reasons, "samples": len(rows)}
+        if note:
+            out["note"] = note
+        return out
 
 
 # --------------------------------------------------------------------------

@@ -25,6 +25,7 @@
 // epilogue (scales, Cin, identity shift) and store the parked tile: the
 // ring keeps draining while a tile is written out.
 #include "gemm.cuh"
+#include "launch_util.cuh"
 #include "profile.cuh"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -534,7 +535,8 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   }
   void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmArgs,
                const long long) = a.single_pass ? gemm_split_kernel<true> : gemm_split_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  static std::atomic<unsigned long long> attr_set[2];
+  cudaError_t e = smem_limit_once(kern, kSmemBytes, attr_set[a.single_pass ? 1 : 0]);
   if (e != cudaSuccess) return e;
   const long long nt = a.B / kTile;
   const long long tpp = a.sym ? nt * (nt + 1) / 2 : nt * nt;

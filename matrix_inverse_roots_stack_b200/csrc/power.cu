@@ -25,6 +25,7 @@
 // The step is bound by HBM: each product reads the split factor once (4
 // bytes per element); the tensor work per byte is small.
 #include "kernels.cuh"
+#include "launch_util.cuh"
 #include "profile.cuh"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -395,7 +396,8 @@ cudaError_t launch_pi_product(const __half* As, const __half* Vt, const float* v
   if (e != cudaSuccess) return e;
   e = encode_f16_3d_map(&mv, Vt, B, kPiStarts, 2ll * nf, kPiStarts);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(pi_product_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+  static std::atomic<unsigned long long> attr_set;
+  e = smem_limit_once(pi_product_kernel, kPSmemBytes, attr_set);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(nf) * static_cast<unsigned>(B / kPRows);
   pi_product_kernel<<<grid, kPThreads, kPSmemBytes, st>>>(ma, mv, v0, W_prev, stats_prev, B, fsize, W_next,

@@ -372,6 +372,9 @@ def main():
         from matrix_inverse_roots_stack_b200 import distributed as sd
         sharded = sd.ShardedShampoo(params, grads, B, make_local=lambda ps, gs: bd.Shampoo(ps, gs, hp=hp, v0=v0))
         live = {"sharded": sharded}
+        g_off = [0]
+        for g in grads:
+            g_off.append(g_off[-1] + g.numel())
         opt = sharded.local
         if opt is None:
             raise SystemExit(f"rank {rank} owns no parameter: use fewer GPUs for this workload")
@@ -391,12 +394,12 @@ def main():
             if "pipe" in live:  # one GPU: copies overlapped with the other groups' work
                 live["pipe"].step(live["hg"], live["hp"])
                 return
-            off = 0
-            for g in grads:
-                n = g.numel()
-                g.view(-1).copy_(host_g[off:off + n], non_blocking=True)
-                off += n
-            live["sharded"].step()
+            # a rank reads only the gradients of the parameters it owns
+            sh = live["sharded"]
+            for i in sh.owned:
+                n = grads[i].numel()
+                grads[i].view(-1).copy_(host_g[g_off[i]:g_off[i] + n], non_blocking=True)
+            sh.step()
             off = 0
             for p in params:
                 n = p.numel()
@@ -509,7 +512,8 @@ def main():
                 t = torch.tensor([e_ms], device=dev)
                 dist.all_reduce(t, op=dist.ReduceOp.MAX)
                 e_ms = float(t.item())
-            e2e = {"value": round(e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 4 * n_g,
+            h2d = 4 * (n_g if world == 1 else sum(grads[i].numel() for i in sharded.owned))
+            e2e = {"value": round(e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": 4 * n_p, **e2e_info}
             del host_g, host_p
         except RuntimeError as exc:

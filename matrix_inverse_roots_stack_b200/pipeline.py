@@ -14,10 +14,22 @@ outside the tensor-core work.  Every block is an independent problem, so the
 grouping does not change the arithmetic of any block.
 """
 
-from typing import List, Optional, Sequence
+from typing import List, Sequence
 
 from . import binding
 from .distributed import partition
+
+
+def parameter_groups(shapes: Sequence[Sequence[int]], B: int, groups: int) -> List[List[int]]:
+    """Indices of the parameters in each group: at most ``groups`` non-empty
+    groups balanced by root cost (greedy, as the multi-GPU ownership), each
+    in increasing index order."""
+    if groups < 1:
+        raise ValueError("groups must be positive")
+    if not shapes:
+        return []
+    owner = partition(shapes, B, min(groups, len(shapes)))
+    return [g for g in ([i for i, o in enumerate(owner) if o == k] for k in range(max(owner) + 1)) if g]
 
 
 class HostPipelinedShampoo:
@@ -32,9 +44,7 @@ class HostPipelinedShampoo:
         self.shapes = [tuple(int(x) for x in s) for s in shapes]
         self.params = [torch.zeros(s, dtype=torch.float32, device=device) for s in self.shapes]
         self.grads = [torch.zeros(s, dtype=torch.float32, device=device) for s in self.shapes]
-        owner = partition(self.shapes, B, max(1, min(groups, len(self.shapes))))
-        self.groups: List[List[int]] = [g for g in ([i for i, o in enumerate(owner) if o == k]
-                                                   for k in range(max(owner) + 1)) if g]
+        self.groups = parameter_groups(self.shapes, B, groups)
         self.opts = [binding.Shampoo([self.params[i] for i in g], [self.grads[i] for i in g], hp=self.hp, v0=v0)
                      for g in self.groups]
         dev = self.params[0].device

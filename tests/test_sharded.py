@@ -42,6 +42,24 @@ def test_partition_is_a_balanced_deterministic_assignment():
         sd.partition([(4, 4)], 128, 0)
 
 
+def test_pipeline_groups_cover_every_parameter_once():
+    from matrix_inverse_roots_stack_b200.pipeline import parameter_groups
+    shapes = workloads.llama_1b_shapes()
+    for groups in (1, 2, 4, 8):
+        gs = parameter_groups(shapes, 1024, groups)
+        assert len(gs) == groups and all(gs)
+        assert sorted(i for g in gs for i in g) == list(range(len(shapes)))
+        assert all(g == sorted(g) for g in gs)
+        # balanced by root cost like the multi-GPU ownership
+        load = [sum(sd.root_cost(shapes[i], 1024) for i in g) for g in gs]
+        assert max(load) <= sum(load) / groups + max(sd.root_cost(s, 1024) for s in shapes)
+    # two parameters, five groups asked: two groups, the costlier parameter first
+    assert parameter_groups([(4, 4), (8, 8)], 128, 5) == [[1], [0]]
+    assert parameter_groups([], 128, 3) == []
+    with pytest.raises(ValueError):
+        parameter_groups([(4, 4)], 128, 0)
+
+
 def test_partition_greedy_order_small_case():
     # costs (B = 4): 4x4 -> 2*64 = 128, 8x4 -> 2*(64+64) = 256, 2x2 -> 16
     shapes = [(4, 4), (8, 4), (2, 2), (4, 4)]

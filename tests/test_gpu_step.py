@@ -86,16 +86,18 @@ def compare(gpu, thetas, grads, hp, steps=1, seed=0):
             br, bc = L.shape[0], R.shape[0]
             assert rel(gpu["factors"][s][2 * k][:br, :br], L) < FACTOR_TOL
             assert rel(gpu["factors"][s][2 * k + 1][:bc, :bc], R) < FACTOR_TOL
+    def close(got, ref, tol):
+        # relative error, or exact agreement where the reference is zero
+        return np.all(got == 0.0) if np.linalg.norm(ref) == 0 else rel(got, ref) < tol
+
     for i, t0 in enumerate(thetas):
         d_gpu = gpu["theta"][i] - t0.astype(np.float64)
         d_ref = th[i] - t0.astype(np.float64)
-        assert rel(d_gpu, d_ref) < UPDATE_TOL, (i, rel(d_gpu, d_ref))
-        assert rel(gpu["m"][i], state["params"][i]["m"]) < MOMENT_TOL
-        assert rel(gpu["v"][i], state["params"][i]["v"]) < MOMENT_TOL
+        assert close(d_gpu, d_ref, UPDATE_TOL), (i, rel(d_gpu, d_ref))
+        assert close(gpu["m"][i], state["params"][i]["m"], MOMENT_TOL)
+        assert close(gpu["v"][i], state["params"][i]["v"], MOMENT_TOL)
         for (r0, r1, c0, c1) in ostep.block_grid(*t0.shape, B):
-            db = d_ref[r0:r1, c0:c1]
-            if np.linalg.norm(db) > 0:
-                assert rel(d_gpu[r0:r1, c0:c1], db) < UPDATE_TOL
+            assert close(d_gpu[r0:r1, c0:c1], d_ref[r0:r1, c0:c1], UPDATE_TOL), (i, r0, c0)
 
 
 def check_lambdas(gpu, grads, hp):
@@ -138,6 +140,25 @@ def test_ragged_edges_multi_param(torch):
               for (r0, r1, c0, c1) in ostep.block_grid(*s, 128)]
     assert [tuple(r[:5]) for r in tab] == expect
     check_lambdas(gpu, grads, hp)  # factors of 44, 8, 5, 7, 64 and 4 inside 128-padded storage
+    compare(gpu, th, grads, hp)
+
+
+def test_zero_gradient_blocks(torch):
+    # a block whose gradient is zero has U_b = 0, hence s_b = 0 and no update
+    # (its factors stay at the initial scaled identity); a parameter whose
+    # whole gradient is zero is not moved at all
+    shapes = [(256, 256), (64, 96)]
+    gs = workloads.gaussian_gradients(shapes, std=0.1, seed=7)
+    gs[0][128:, :128] = 0.0
+    gs[1][:] = 0.0
+    grads = [[g] for g in gs]
+    th = workloads.parameters(shapes, seed=8)
+    hp = ostep.HParams(block_size=128, ndb_iters1=12, ndb_iters2=12)
+    gpu = run_gpu(torch, th, grads, hp)
+    d0 = gpu["theta"][0] - th[0].astype(np.float64)
+    assert np.all(d0[128:, :128] == 0.0)
+    assert np.all(gpu["theta"][1] == th[1].astype(np.float64))
+    check_lambdas(gpu, grads, hp)
     compare(gpu, th, grads, hp)
 
 

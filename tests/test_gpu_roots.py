@@ -106,7 +106,8 @@ def test_ndb_many_tiles(torch):
         assert rel(X[i], r) < ROOT_TOL, (i, rel(X[i], r))
 
 
-@pytest.mark.parametrize("d,delta", [(2, 1e-3), (3, 1e-3), (16, 1e-3), (16, 1e-6), (40, 1e-3)])
+# degree 60 is the explainer's "degree ~60" ("Building blocks", Chebyshev)
+@pytest.mark.parametrize("d,delta", [(2, 1e-3), (3, 1e-3), (16, 1e-3), (16, 1e-6), (40, 1e-3), (60, 1e-3)])
 def test_chebyshev(torch, d, delta):
     A = workloads.spd_stack_geometric(4, 256, 1e3, seed=5)
     X, lam, rc, v0 = gpu_roots(torch, A, "cheb", degree=d, delta=delta, eps=1e-6)

@@ -38,6 +38,12 @@
  *    exception crosses this boundary.  On an error return nothing has been
  *    enqueued unless the code is SHAMPOO_ECUDA.
  *  - A ctx is not thread-safe; use one ctx per stream.
+ *  - CUDA graphs: after a first call on a device (which sets the kernels'
+ *    shared-memory limits), the standalone root calls make only stream-
+ *    ordered CUDA calls, so a call can be captured and replayed with new
+ *    inputs in the same buffers.  shampoo_precondition_step bakes its step
+ *    number (Adam bias correction, root reuse) into the launches: capture it
+ *    per step value or call it eagerly.
  */
 #ifndef DASH_B200_H
 #define DASH_B200_H

@@ -41,9 +41,9 @@
  *  - CUDA graphs: after a first call on a device (which sets the kernels'
  *    shared-memory limits), the standalone root calls make only stream-
  *    ordered CUDA calls, so a call can be captured and replayed with new
- *    inputs in the same buffers.  shampoo_precondition_step bakes its step
- *    number (Adam bias correction, root reuse) into the launches: capture it
- *    per step value or call it eagerly.
+ *    inputs in the same buffers.  So can a full step (shampoo_accumulate +
+ *    shampoo_precondition_step with step = 0, which takes its step number
+ *    from a counter on the device), after one eager step on the same ws.
  */
 #ifndef DASH_B200_H
 #define DASH_B200_H
@@ -164,6 +164,11 @@ SHAMPOO_API int shampoo_accumulate(shampoo_ctx* ctx, float* factors, void* ws, s
  * with the roots kept in ws since the last root step (the factors, moments
  * and parameters are still updated every step), and leave lambda_out and
  * roots_out untouched.
+ * `step` >= 1 is the step number; it also sets a step counter kept in ws.
+ * `step` = 0 continues that counter on the device (t = previous t + 1), so
+ * that a captured step can be replayed from a CUDA graph; it requires
+ * root_every <= 1 (roots every step) and an earlier call with an explicit
+ * step on the same ws, else SHAMPOO_EINVAL.  step < 0: SHAMPOO_EINVAL.
  * `lambda_out` (device, n_factors floats, or NULL) receives the estimates.
  * `roots_out` (device, (n_factors, B, B) fp32, or NULL) receives X. */
 SHAMPOO_API int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const float* v0, int step,

@@ -278,17 +278,20 @@ class Shampoo:
         _check(load().shampoo_accumulate(self._ctx, _ptr(self.factors), _ptr(self.ws), self.ws.numel(),
                                          _stream(stream)), "shampoo_accumulate")
 
-    def precondition_step(self, roots_out=None, stream=None):
+    def precondition_step(self, roots_out=None, stream=None, device_step=False):
+        """device_step: take the step number from the counter on the device
+        (for steps captured into a CUDA graph; needs an earlier eager step)."""
         self.t += 1
-        _check(load().shampoo_precondition_step(self._ctx, _ptr(self.factors), _ptr(self.v0), self.t,
+        _check(load().shampoo_precondition_step(self._ctx, _ptr(self.factors), _ptr(self.v0),
+                                                0 if device_step else self.t,
                                                 _ptr(self.lam), _ptr(roots_out), _ptr(self.ws),
                                                 self.ws.numel(), _stream(stream)),
                "shampoo_precondition_step")
 
-    def step(self, roots_out=None, stream=None):
+    def step(self, roots_out=None, stream=None, device_step=False):
         """One full step: factor EMA, roots, precondition, Adam graft, update."""
         self.accumulate(stream)
-        self.precondition_step(roots_out, stream)
+        self.precondition_step(roots_out, stream, device_step)
 
     def status(self, stream=None):
         return read_status(self.ws, stream)

@@ -471,9 +471,10 @@ struct shampoo_ctx {
   int n_blocks = 0, n_factors = 0;
   RootLayout roots{};
   size_t off_gs = 0, off_roots = 0, off_u = 0, off_pn = 0, off_un = 0, off_blocks = 0, off_params = 0,
-         off_prefix = 0, off_fsize = 0, total = 0;
+         off_prefix = 0, off_fsize = 0, off_step = 0, total = 0;
   const void* tables_ws = nullptr;
   const void* roots_ws = nullptr;  // workspace holding the roots of the last root step
+  const void* step_ws = nullptr;   // workspace whose step counter an explicit step has set
 };
 
 namespace {
@@ -595,6 +596,7 @@ int shampoo_init_blocks(shampoo_ctx** out, const shampoo_param* params, int n_pa
   c->off_params = b.take(sizeof(ParamDev) * n_params);
   c->off_prefix = b.take(sizeof(long long) * (n_params + 1));
   c->off_fsize = b.take(sizeof(int) * c->n_factors);
+  c->off_step = b.take(4 * sizeof(int));  // step counter and the Adam bias corrections
   c->total = b.off;
   *workspace_bytes = c->total;
   *out = c;
@@ -665,9 +667,12 @@ int shampoo_accumulate(shampoo_ctx* ctx, float* factors, void* ws_v, size_t ws_b
 
 int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const float* v0, int step, float* lambda_out,
                               float* roots_out, void* ws_v, size_t ws_bytes, void* stream) {
-  if (!ctx || !factors || !v0 || step < 1) return SHAMPOO_EINVAL;
+  if (!ctx || !factors || !v0 || step < 0) return SHAMPOO_EINVAL;
   int rc = check_ws(ws_v, ws_bytes, ctx->total);
   if (rc) return rc;
+  // step 0 continues the device step counter: the roots are then recomputed
+  // every step, and an explicit step must have set the counter first
+  if (step == 0 && ((ctx->hp.root_every > 1) || ctx->step_ws != ws_v)) return SHAMPOO_EINVAL;
   char* ws = static_cast<char*>(ws_v);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = upload_tables(ctx, ws, st);
@@ -678,7 +683,7 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   const int* fsize = reinterpret_cast<const int*>(ws + ctx->off_fsize);
   __half* roots = split_at(ws, ctx->off_roots, 0, B);
   const int every = hp.root_every > 0 ? hp.root_every : 1;
-  if ((step - 1) % every == 0 || ctx->roots_ws != ws_v) {  // root step (or no roots kept in this ws yet)
+  if (step == 0 || (step - 1) % every == 0 || ctx->roots_ws != ws_v) {  // root step (or no roots kept yet)
     const int pi = hp.scaling == SHAMPOO_SCALING_FROBENIUS ? 0 : hp.pi_iters;
     const bool cn = hp.solver == SHAMPOO_SOLVER_COUPLED_NEWTON;
     rc = run_roots(factors, nf, B, hp.eps, fsize, v0, pi, hp.solver, cn ? hp.cn_iters : hp.ndb_iters1,
@@ -724,13 +729,14 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   }
   dash::prof_end(uslot, st);
   const int dslot = dash::prof_begin(dash::kProfAdam, st);
-  const double bc1 = 1.0 - std::pow(static_cast<double>(hp.beta1), step);
-  const double bc2 = 1.0 - std::pow(static_cast<double>(hp.beta2), step);
   const ParamDev* pd = reinterpret_cast<const ParamDev*>(ws + ctx->off_params);
   const long long* prefix = reinterpret_cast<const long long*>(ws + ctx->off_prefix);
   const int np = static_cast<int>(ctx->params.size());
-  dash::launch_adam(pd, prefix, np, ctx->n_items, B, hp.beta1, hp.beta2, hp.adam_eps, static_cast<float>(bc1),
-                    static_cast<float>(bc2), pn, st);
+  int* info = reinterpret_cast<int*>(ws + ctx->off_step);
+  dash::launch_step_info(info, step, hp.beta1, hp.beta2, st);
+  DASH_LAUNCHED();
+  if (step > 0) ctx->step_ws = ws_v;
+  dash::launch_adam(pd, prefix, np, ctx->n_items, B, hp.beta1, hp.beta2, hp.adam_eps, info, pn, st);
   DASH_LAUNCHED();
   dash::launch_update(pd, prefix, np, ctx->n_items, B, hp.lr, U, pn, un, st);
   DASH_LAUNCHED();

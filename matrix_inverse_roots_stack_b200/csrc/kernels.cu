@@ -257,10 +257,22 @@ __device__ __forceinline__ void adam4(const float* g, float* m, float* v, float 
   }
 }
 
+// The step's Adam bias corrections on the device: step > 0 sets the step
+// counter info[0] to it; step == 0 advances the counter by one.  info[1],
+// info[2] receive 1 / (1 - beta1^t) and 1 / (1 - beta2^t) as floats.
+__global__ void step_info_kernel(int* __restrict__ info, int step, float beta1, float beta2) {
+  const int t = step > 0 ? step : info[0] + 1;
+  info[0] = t;
+  float* f = reinterpret_cast<float*>(info + 1);
+  f[0] = 1.0f / static_cast<float>(1.0 - pow(static_cast<double>(beta1), t));
+  f[1] = 1.0f / static_cast<float>(1.0 - pow(static_cast<double>(beta2), t));
+}
+
 __global__ void __launch_bounds__(256) adam_kernel(const ParamDev* __restrict__ params,
                                                    const long long* __restrict__ prefix, int n_params, int B,
-                                                   float b1, float b2, float eps, float ibc1, float ibc2,
+                                                   float b1, float b2, float eps, const int* __restrict__ info,
                                                    float* __restrict__ pnorm) {
+  const float ibc1 = __int_as_float(info[1]), ibc2 = __int_as_float(info[2]);
   __shared__ float wsum[8];
   __shared__ int wblk[8];
   const long long item = blockIdx.x;
@@ -415,10 +427,15 @@ void launch_init_factors(float* F, int nf, int B, float init_scale, cudaStream_t
   prof_count_launch();
 }
 
+void launch_step_info(int* info, int step, float beta1, float beta2, cudaStream_t st) {
+  step_info_kernel<<<1, 1, 0, st>>>(info, step, beta1, beta2);
+  prof_count_launch();
+}
+
 void launch_adam(const ParamDev* params, const long long* item_prefix, int n_params, long long n_items, int B,
-                 float beta1, float beta2, float adam_eps, float bc1, float bc2, float* pnorm, cudaStream_t st) {
+                 float beta1, float beta2, float adam_eps, const int* info, float* pnorm, cudaStream_t st) {
   adam_kernel<<<static_cast<unsigned>(n_items), 256, 0, st>>>(params, item_prefix, n_params, B, beta1, beta2,
-                                                               adam_eps, 1.0f / bc1, 1.0f / bc2, pnorm);
+                                                               adam_eps, info, pnorm);
   prof_count_launch();
 }
 

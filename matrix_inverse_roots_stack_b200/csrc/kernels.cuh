@@ -93,9 +93,15 @@ void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int 
 // factors[f] = init_scale * I.
 void launch_init_factors(float* F, int nf, int B, float init_scale, cudaStream_t st);
 
-// Adam moments and per-block sum of squares of the Adam direction P.
+// Step counter and Adam bias corrections on the device: info[0] = step if
+// step > 0, else info[0] + 1; info[1], info[2] = 1 / (1 - beta1^t),
+// 1 / (1 - beta2^t) (float bits).
+void launch_step_info(int* info, int step, float beta1, float beta2, cudaStream_t st);
+
+// Adam moments and per-block sum of squares of the Adam direction P, with
+// the bias corrections of launch_step_info's info.
 void launch_adam(const ParamDev* params, const long long* item_prefix, int n_params, long long n_items, int B,
-                 float beta1, float beta2, float adam_eps, float bc1, float bc2, float* pnorm, cudaStream_t st);
+                 float beta1, float beta2, float adam_eps, const int* info, float* pnorm, cudaStream_t st);
 
 // param -= lr * sqrt(pnorm_k / unorm_k) * U (0 where unorm_k == 0).
 void launch_update(const ParamDev* params, const long long* item_prefix, int n_params, long long n_items, int B,

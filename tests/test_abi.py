@@ -157,5 +157,9 @@ def test_step_calls_validate_workspace(lib):
                                          None) == bd.SHAMPOO_EINVAL
     assert lib.shampoo_precondition_step(ctx, p, None, 1, None, None, ctypes.c_void_p(0x100000), nbytes,
                                          None) == bd.SHAMPOO_EINVAL
+    # step 0 continues the device step counter: not before an explicit step on
+    # this workspace (the call above returned before setting it), never below 0
+    assert lib.shampoo_precondition_step(ctx, p, p, -1, None, None, ctypes.c_void_p(0x100000), nbytes,
+                                         None) == bd.SHAMPOO_EINVAL
     lib.shampoo_destroy(ctx)
     lib.shampoo_destroy(None)

@@ -68,3 +68,51 @@ def test_standalone_roots_replay_from_a_cuda_graph(torch, solver):
         assert rel(lam.cpu().numpy(), le.cpu().numpy()) < 1e-5, (solver, name)
         for i in range(n):
             assert rel(X[i].cpu().numpy(), Xe[i].cpu().numpy()) < 1e-5, (solver, name, i)
+
+
+def test_full_step_replays_from_a_cuda_graph(torch):
+    # after one eager step, a step whose number comes from the device counter
+    # (step = 0 at the C ABI) is captured once and replayed for the later
+    # steps; it must match a twin optimizer stepped eagerly with explicit
+    # step numbers (Adam bias correction included)
+    from matrix_inverse_roots_stack_b200 import binding as bd
+    shapes = [(300, 200), (128, 256), (5, 7)]
+    B = 128
+    hp = bd.make_hparams(block_size=B, ndb_iters1=12, ndb_iters2=12)
+    v0 = torch.from_numpy(workloads.pi_start_vectors(B, 32, seed=0)).cuda()
+    theta = workloads.parameters(shapes, seed=2)
+    steps = [workloads.gaussian_gradients(shapes, std=0.1, seed=20 + k) for k in range(4)]
+
+    def make():
+        P = [torch.from_numpy(t.copy()).cuda() for t in theta]
+        G = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes]
+        return P, G, bd.Shampoo(P, G, hp=hp, v0=v0)
+
+    def load(G, gs):
+        for g, x in zip(G, gs):
+            g.copy_(torch.from_numpy(x))
+
+    Pe, Ge, ref = make()
+    for gs in steps:
+        load(Ge, gs)
+        ref.step()
+    Pg, Gg, opt = make()
+    load(Gg, steps[0])
+    opt.step()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        opt.step(device_step=True)
+    for gs in steps[1:]:
+        load(Gg, gs)
+        g.replay()
+    torch.cuda.synchronize()
+    assert ref.status()[0] == 0 and opt.status()[0] == 0
+    for i in range(len(shapes)):
+        d_ref = Pe[i].cpu().numpy().astype(np.float64) - theta[i]
+        d_got = Pg[i].cpu().numpy().astype(np.float64) - theta[i]
+        assert rel(d_got, d_ref) < 1e-5, i
+        assert rel(opt.m[i].cpu().numpy(), ref.m[i].cpu().numpy()) < 1e-6, i
+        assert rel(opt.v[i].cpu().numpy(), ref.v[i].cpu().numpy()) < 1e-6, i

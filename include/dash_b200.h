@@ -20,7 +20,8 @@
  *  - B (the block size) must be a multiple of 128 in [128, 2048].
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Device work is enqueued on it asynchronously; no call
- *    synchronises except shampoo_read_status.
+ *    synchronises except the three status readers (shampoo_read_status,
+ *    shampoo_get_status, shampoo_read_static_status).
  *  - `ws` is a caller-owned device workspace of at least the size the
  *    matching *_workspace_bytes call reports, 256-byte aligned.  Its first
  *    word is a status word that every call clears when it starts and that the
@@ -192,12 +193,14 @@ SHAMPOO_API int shampoo_inv_root_newton_db(const float* A, float* X, int n, int 
                                void* stream);
 
 /* Standalone inverse fourth roots of a stack, Chebyshev solver ("Building
- * blocks", Chebyshev; "Step-by-step", solver (d)): the spectrum of
- * A_i' = A_i + eps I is mapped into [delta, 1 + delta] by A_i'/lambda_i +
- * delta I; p of degree `degree` interpolates x^(-1/4) at the first-kind
- * Chebyshev nodes of that interval (fitted on the host in double precision);
- * p is evaluated with the matrix Clenshaw recurrence; X_i = lambda_i^(-1/4) p
- * ~ (A_i' + delta lambda_i I)^(-1/4).  Arguments as for the Newton-DB call. */
+ * blocks", Chebyshev; "Step-by-step", solver (d)): A_i' = A_i + eps I;
+ * lambda_i as for the Newton-DB call; the common spectral scaling
+ * c = 1/(2 lambda_i) of "Step-by-step" maps the spectrum of A_i' into
+ * [delta, 1 + delta] by x = c A_i' + delta I (t = 2 c A_i' - I on [-1, 1]);
+ * p of degree `degree` interpolates x^(-1/4) at the first-kind Chebyshev
+ * nodes of [delta, 1 + delta] (fitted on the host in double precision); p is
+ * evaluated with the matrix Clenshaw recurrence in t; X_i = c^(1/4) p(x)
+ * ~ (A_i' + 2 delta lambda_i I)^(-1/4).  Arguments as for the Newton-DB call. */
 SHAMPOO_API int shampoo_inv_root_chebyshev(const float* A, float* X, int n, int B, int degree, float delta, float eps,
                                const float* v0, int pi_iters, float* lambda_out, void* ws, size_t ws_bytes,
                                void* stream);
@@ -225,24 +228,33 @@ SHAMPOO_API int shampoo_inv_root_coupled_newton(const float* A, float* X, int n,
  * library's device global memory; every GPU that loads the library holds it
  * until the process exits.  Problems whose workspace
  * (shampoo_inv_root_workspace_bytes(n, B, SHAMPOO_SOLVER_NEWTON_DB)) exceeds it
- * are rejected with SHAMPOO_EWORKSPACE (it holds up to 168 matrices of 128,
- * 47 of 256, 12 of 512, 3 of 1024).  The caller still passes A, X, v0 and lambda_out (device
+ * are rejected with SHAMPOO_EWORKSPACE (it holds up to 161 matrices of 128,
+ * 46 of 256, 12 of 512, 3 of 1024).  The caller still passes A, X, v0 and lambda_out (device
  * pointers, as for shampoo_inv_root_newton_db); the computation and the
  * results are the same.
  *
- * The first call on a device looks up the scratch's device address (once per
- * device, with that device current); make that first call before any stream
+ * Every call looks up the scratch's device address with the caller's device
+ * current (an address kept across calls could go stale if the device's
+ * context were torn down); the first call on a device also loads the
+ * library's device code there, so make that first call before any stream
  * capture.  All calls share the one array and it keeps the last call's
  * contents (each call clears what must start at zero), so calls whose GPU work
  * overlaps -- on different streams, or from different threads -- race on it:
- * serialise them.  The status word lives in the scratch too and is cleared at
- * each call; it is not readable through this entry point.
+ * serialise them.  The status word (non-finite values, a bounded wait that
+ * gave up) lives in the scratch too; each call clears it, and
+ * shampoo_read_static_status reads it.
  * Errors: as shampoo_inv_root_newton_db, plus SHAMPOO_EWORKSPACE when the
  * problem does not fit the scratch. */
 #define SHAMPOO_STATIC_SCRATCH_BYTES (64u << 20)
 SHAMPOO_API int shampoo_inv_root_newton_db_static(const float* A, float* X, int n, int B, int iters1, int iters2,
                                                   float eps, const float* v0, int pi_iters, float* lambda_out,
                                                   void* stream);
+
+/* Status word of the static scratch after shampoo_inv_root_newton_db_static
+ * (no counterpart in the paper): synchronises `stream`, reads the word into
+ * *flags (host, may be NULL) and returns as shampoo_read_status does.  It
+ * reports the last static call whose work has finished on this device. */
+SHAMPOO_API int shampoo_read_static_status(void* stream, unsigned* flags);
 
 /* Workspace bytes for a standalone root call on n matrices of size B. */
 SHAMPOO_API size_t shampoo_inv_root_workspace_bytes(int n, int B, int solver);
@@ -251,6 +263,13 @@ SHAMPOO_API size_t shampoo_inv_root_workspace_bytes(int n, int B, int solver);
  * be NULL) and return SHAMPOO_OK, SHAMPOO_ETIMEOUT (checked first: a wait
  * that gave up leaves later results undefined) or SHAMPOO_ENONFINITE. */
 SHAMPOO_API int shampoo_read_status(const void* ws, void* stream, unsigned* flags);
+
+/* Status of a ctx's last step: synchronises the stream that the last
+ * shampoo_accumulate or shampoo_precondition_step on `ctx` was given, reads
+ * the status word of that call's workspace into *device_flags (host, may be
+ * NULL; SHAMPOO_STATUS_* bits) and returns as shampoo_read_status does.
+ * Before any step call it reports 0 and SHAMPOO_OK. */
+SHAMPOO_API int shampoo_get_status(shampoo_ctx* ctx, int* device_flags);
 
 /* Static description of a status code. */
 SHAMPOO_API const char* shampoo_strerror(int code);

@@ -74,6 +74,8 @@ _PROTOS = {
     "shampoo_inv_root_coupled_newton": (_I, [_VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _VP, _VP, _SZ, _VP]),
     "shampoo_inv_root_workspace_bytes": (_SZ, [_I, _I, _I]),
     "shampoo_read_status": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_uint)]),
+    "shampoo_read_static_status": (_I, [_VP, ctypes.POINTER(ctypes.c_uint)]),
+    "shampoo_get_status": (_I, [_VP, ctypes.POINTER(ctypes.c_int)]),
     "shampoo_strerror": (ctypes.c_char_p, [_I]),
     "shampoo_destroy": (None, [_VP]),
     "shampoo_inv_root_newton_db_static": (_I, [_VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _VP, _VP]),
@@ -209,6 +211,14 @@ def read_status(ws, stream=None):
     return rc, flags.value
 
 
+def read_static_status(stream=None):
+    """(code, flags) of the static scratch's status word (after
+    :func:`inv_root_newton_db_static`)."""
+    flags = ctypes.c_uint(0)
+    rc = load().shampoo_read_static_status(_stream(stream), ctypes.byref(flags))
+    return rc, flags.value
+
+
 PROFILE_STAGES = ("gemm", "accumulate", "power_iteration", "solver", "precondition", "adam_update")
 
 
@@ -295,6 +305,13 @@ class Shampoo:
 
     def status(self, stream=None):
         return read_status(self.ws, stream)
+
+    def get_status(self):
+        """(code, flags) of the last step call's workspace, on the stream it
+        was given (the library remembers both)."""
+        flags = ctypes.c_int(0)
+        rc = load().shampoo_get_status(self._ctx, ctypes.byref(flags))
+        return rc, flags.value
 
     def __del__(self):
         ctx = getattr(self, "_ctx", None)

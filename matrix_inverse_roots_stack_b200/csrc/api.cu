@@ -19,6 +19,10 @@ using dash::BlockDesc;
 using dash::GemmArgs;
 using dash::ParamDev;
 
+namespace dash {
+int read_status_word(const void* ws, void* stream, unsigned* flags);
+}
+
 namespace {
 
 constexpr float kZScale = 16.0f;  // Newton-DB Z is stored divided by this (fp16 range headroom)
@@ -475,6 +479,8 @@ struct shampoo_ctx {
   const void* tables_ws = nullptr;
   const void* roots_ws = nullptr;  // workspace holding the roots of the last root step
   const void* step_ws = nullptr;   // workspace whose step counter an explicit step has set
+  const void* last_ws = nullptr;   // workspace and stream of the last step call (shampoo_get_status)
+  void* last_stream = nullptr;
 };
 
 namespace {
@@ -641,6 +647,8 @@ int shampoo_accumulate(shampoo_ctx* ctx, float* factors, void* ws_v, size_t ws_b
   if (rc) return rc;
   char* ws = static_cast<char*>(ws_v);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_ws = ws_v;
+  ctx->last_stream = stream;
   rc = upload_tables(ctx, ws, st);
   if (rc) return rc;
   unsigned* status = reinterpret_cast<unsigned*>(ws + ctx->roots.status);
@@ -675,6 +683,8 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   if (step == 0 && ((ctx->hp.root_every > 1) || ctx->step_ws != ws_v)) return SHAMPOO_EINVAL;
   char* ws = static_cast<char*>(ws_v);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ctx->last_ws = ws_v;
+  ctx->last_stream = stream;
   rc = upload_tables(ctx, ws, st);
   if (rc) return rc;
   const shampoo_hparams& hp = ctx->hp;
@@ -735,11 +745,12 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
   int* info = reinterpret_cast<int*>(ws + ctx->off_step);
   dash::launch_step_info(info, step, hp.beta1, hp.beta2, st);
   DASH_LAUNCHED();
-  if (step > 0) ctx->step_ws = ws_v;
   dash::launch_adam(pd, prefix, np, ctx->n_items, B, hp.beta1, hp.beta2, hp.adam_eps, info, pn, st);
   DASH_LAUNCHED();
   dash::launch_update(pd, prefix, np, ctx->n_items, B, hp.lr, U, pn, un, st);
   DASH_LAUNCHED();
+  // only a step whose launches were all queued may be continued by step 0
+  if (step > 0) ctx->step_ws = ws_v;
   dash::prof_end(dslot, st);
   return SHAMPOO_OK;
 }
@@ -798,15 +809,20 @@ int shampoo_inv_root_coupled_newton(const float* A, float* X, int n, int B, int 
 }
 
 int shampoo_read_status(const void* ws, void* stream, unsigned* flags) {
-  if (!ws) return SHAMPOO_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DASH_TRY(cudaStreamSynchronize(st));
+  return dash::read_status_word(ws, stream, flags);
+}
+
+int shampoo_get_status(shampoo_ctx* ctx, int* device_flags) {
+  if (!ctx) return SHAMPOO_EINVAL;
+  if (!ctx->last_ws) {  // no step call has run on this ctx yet: nothing to report
+    if (device_flags) *device_flags = 0;
+    return SHAMPOO_OK;
+  }
   unsigned w = 0;
-  DASH_TRY(cudaMemcpy(&w, ws, sizeof(unsigned), cudaMemcpyDeviceToHost));
-  if (flags) *flags = w;
-  if (w & dash::kStatusTimeout) return SHAMPOO_ETIMEOUT;  // the root cause when both are set
-  if (w & dash::kStatusNonFinite) return SHAMPOO_ENONFINITE;
-  return SHAMPOO_OK;
+  const int rc = dash::read_status_word(static_cast<const char*>(ctx->last_ws) + ctx->roots.status,
+                                        ctx->last_stream, &w);
+  if (device_flags) *device_flags = static_cast<int>(w);
+  return rc;
 }
 
 const char* shampoo_strerror(int code) {
@@ -832,6 +848,19 @@ int shampoo_debug_inject_timeout(void) {
 }  // extern "C"
 
 namespace dash {
+
+// Synchronise the stream and read a status word (shared by the status calls).
+int read_status_word(const void* ws, void* stream, unsigned* flags) {
+  if (!ws) return SHAMPOO_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DASH_TRY(cudaStreamSynchronize(st));
+  unsigned w = 0;
+  DASH_TRY(cudaMemcpy(&w, ws, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  if (flags) *flags = w;
+  if (w & dash::kStatusTimeout) return SHAMPOO_ETIMEOUT;  // the root cause when both are set
+  if (w & dash::kStatusNonFinite) return SHAMPOO_ENONFINITE;
+  return SHAMPOO_OK;
+}
 
 // Standalone root computation on a caller-provided scratch region (used by
 // the static-scratch entry point in noalloc.cu).

@@ -1,8 +1,6 @@
 // Newton-DB inverse fourth roots with library-owned scratch, for callers that
 // cannot allocate device memory themselves (see shampoo_inv_root_newton_db_static
 // in include/dash_b200.h).
-#include <mutex>
-
 #include <cuda_runtime.h>
 
 #include "dash_b200.h"
@@ -11,6 +9,7 @@ namespace dash {
 int inv_root_with_scratch(const float* A, float* X, int n, int B, float eps, const float* v0, int pi_iters, void* ws,
                           size_t ws_bytes, int solver, int it1, int it2, int degree, float delta, float* lambda_out,
                           void* stream);
+int read_status_word(const void* ws, void* stream, unsigned* flags);
 }
 
 namespace {
@@ -19,25 +18,17 @@ namespace {
 // module's global memory, so each GPU that loads this library keeps it
 // (SHAMPOO_STATIC_SCRATCH_BYTES) until the process exits.  In host code this
 // name is only a host-side stand-in: kernels are given the device address
-// obtained below.
+// obtained below.  The root layout puts the status word at offset 0.
 __device__ __align__(256) unsigned char g_static_scratch[SHAMPOO_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device, looked up once per
-// device (the first call on a device does this set-up).
+// Device address of the scratch on the current device.  It is looked up on
+// every call, with the caller's device current: an address kept from an
+// earlier call could be stale after the device's context was torn down and
+// the module loaded again.  The first call on a device also loads the module.
 int scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SHAMPOO_ECUDA;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SHAMPOO_ECUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SHAMPOO_ECUDA;
+  *out = p;
   return SHAMPOO_OK;
 }
 
@@ -58,6 +49,13 @@ SHAMPOO_API int shampoo_inv_root_newton_db_static(const float* A, float* X, int 
   if (rc) return rc;
   return dash::inv_root_with_scratch(A, X, n, B, eps, v0, pi_iters, ws, SHAMPOO_STATIC_SCRATCH_BYTES,
                                      SHAMPOO_SOLVER_NEWTON_DB, iters1, iters2, 0, 0.0f, lambda_out, stream);
+}
+
+SHAMPOO_API int shampoo_read_static_status(void* stream, unsigned* flags) {
+  void* ws = nullptr;
+  const int rc = scratch_address(&ws);
+  if (rc) return rc;
+  return dash::read_status_word(ws, stream, flags);
 }
 
 }  // extern "C"

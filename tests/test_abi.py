@@ -163,3 +163,42 @@ def test_step_calls_validate_workspace(lib):
                                          None) == bd.SHAMPOO_EINVAL
     lib.shampoo_destroy(ctx)
     lib.shampoo_destroy(None)
+
+
+def test_header_static_capacity_matches_layout(lib):
+    """The capacities the header states for the static scratch are the
+    largest stacks whose workspace fits SHAMPOO_STATIC_SCRATCH_BYTES."""
+    text = open(os.path.join(HEADER_DIR, "dash_b200.h")).read()
+    flat = " ".join(text.split()).replace(" * ", " ")
+    m = re.search(r"holds up to (\d+) matrices of 128, (\d+) of 256, (\d+) of 512, (\d+) of 1024", flat)
+    assert m, "capacity sentence missing from the header"
+    cap = re.search(r"#define SHAMPOO_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    scratch = int(cap.group(1)) << int(cap.group(2))
+    assert scratch == bd.STATIC_SCRATCH_BYTES
+    for B, stated in zip((128, 256, 512, 1024), map(int, m.groups())):
+        fits = lambda n: lib.shampoo_inv_root_workspace_bytes(n, B, bd.SOLVER_NEWTON_DB) <= scratch
+        assert fits(stated) and not fits(stated + 1), (B, stated)
+
+
+def test_header_codes_and_chebyshev_contract():
+    text = open(os.path.join(HEADER_DIR, "dash_b200.h")).read()
+    codes = dict(re.findall(r"#define (SHAMPOO_E\w+|SHAMPOO_OK) \(?(-?\d+)\)?", text))
+    assert {k: int(v) for k, v in codes.items()} == {
+        "SHAMPOO_OK": bd.SHAMPOO_OK, "SHAMPOO_EINVAL": bd.SHAMPOO_EINVAL,
+        "SHAMPOO_EUNSUPPORTED": bd.SHAMPOO_EUNSUPPORTED, "SHAMPOO_EWORKSPACE": bd.SHAMPOO_EWORKSPACE,
+        "SHAMPOO_ECUDA": bd.SHAMPOO_ECUDA, "SHAMPOO_ENONFINITE": bd.SHAMPOO_ENONFINITE,
+        "SHAMPOO_ETIMEOUT": bd.SHAMPOO_ETIMEOUT}
+    flat = " ".join(text.split()).replace(" * ", " ")
+    # the Chebyshev map the kernels and the oracle run: c = 1/(2 lambda),
+    # x = c A' + delta I, X = c^(1/4) p(x) ~ (A' + 2 delta lambda I)^(-1/4)
+    assert "c = 1/(2 lambda_i)" in flat and "x = c A_i' + delta I" in flat
+    assert "X_i = c^(1/4) p(x) ~ (A_i' + 2 delta lambda_i I)^(-1/4)" in flat
+
+
+def test_get_status_before_any_step(lib):
+    rc, ctx, _ = init(lib, [(256, 256)], block_size=128)
+    assert rc == 0
+    flags = ctypes.c_int(7)
+    assert lib.shampoo_get_status(ctx, ctypes.byref(flags)) == bd.SHAMPOO_OK and flags.value == 0
+    assert lib.shampoo_get_status(None, ctypes.byref(flags)) == bd.SHAMPOO_EINVAL
+    lib.shampoo_destroy(ctx)

@@ -197,6 +197,37 @@ def test_cn_matrix_keeps_the_coupling_invariant():
         assert rel(M, np.linalg.matrix_power(X, 4) @ M0) < 1e-12
 
 
+@pytest.mark.parametrize("delta", [1e-2, 1e-3, 1e-4])
+def test_cn_newton_step_contracts_quadratically(delta):
+    # Guo-Higham Newton step for p = 4 near the fixed point: with
+    # m = 1 - delta, C = (5 - m)/4 = 1 + delta/4 and
+    # 1 - C^4 m = (5/8) delta^2 + (5/16) delta^3 + O(delta^4): the constant is
+    # (p + 1)/(2p).  Any other affine C_k (e.g. (3 - m)/2) loses the quadratic
+    # term or changes its constant, and the coupling invariant cannot see it.
+    x, m = roots.cn_scalar(np.array([1.0 - delta]), 1)
+    assert abs(x[0] - (1.0 + delta / 4.0)) < 1e-15
+    ratio = (1.0 - m[0]) / delta ** 2
+    assert abs(ratio - 0.625) < 0.4 * delta, ratio
+
+
+def test_cn_one_and_two_steps_closed_form():
+    # T = 1 and T = 2 written out from the step's definition, on the
+    # eigenvalues of M0 (not through cn_scalar): X1 = C0 = (5I - M0)/4,
+    # M1 = C0^4 M0, X2 = C0 (5I - M1)/4.
+    A, U, w = random_spd(20, 50.0, seed=14)
+    lam = 1.05 * w.max()
+    c = 1.0 / (2.0 * lam)
+    m0 = c * w
+    c0 = (5.0 - m0) / 4.0
+    x1 = c0
+    m1 = c0 ** 4 * m0
+    x2 = c0 * (5.0 - m1) / 4.0
+    for T, x in ((1, x1), (2, x2)):
+        expect = (U * (c ** 0.25 * x)) @ U.T
+        assert rel(roots.cn_inv4root_spectral(A, lam, T), expect) < 1e-13
+        assert rel(roots.cn_inv4root_matmul(A, lam, T), expect) < 1e-12
+
+
 def test_cn_level2_matches_level3():
     A, _, w = random_spd(48, 1e3, seed=12)
     lam = w.max() * 0.999

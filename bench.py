@@ -43,7 +43,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 
 # DRAM bytes (read + write) per executed tensor-core flop of gemm_split_kernel,
 # by (block size, solver): from an ncu capture of every GEMM launch of one step
-# of the mixed-shape B=1024 workload (profiles/gemm_split_kernel_traffic_b1024_ndb14.md).
+# of the mixed-shape B=1024 workload (24 factors of 1024, Newton-DB 14 + 14).
 # Each launch reads and writes its problems' split matrices about once, so a
 # launch's traffic grows in proportion to the problems, and executed flops, it
 # covers; the roofline's per-launch traffic scales this ratio by those flops.
@@ -201,10 +201,16 @@ class ClockSampler:
 # CPU baseline / reference arm: the float64 oracle on a bounded sample
 # --------------------------------------------------------------------------
 
-def oracle_sample(spec, args, budget_s=15.0, seed=0):
-    """Time the oracle step on the first blocks of the workload until about
-    budget_s seconds of CPU work; returns (ms per full step extrapolated by
-    block count, description, threads)."""
+# Blocks of the workload the oracle is timed on (the first parameters, in
+# order, until at least this many blocks): one fixed sample, used by both the
+# cpu_baseline leg and the reference arm, of about 5-15 s of CPU work.
+ORACLE_SAMPLE_BLOCKS = {"llama1b": 40, "gpt2": 60, "spiked512": 16, "mixed": 12, "roots256": 4}
+
+
+def oracle_sample(spec, args, seed=0):
+    """Time the oracle step on a fixed sample of the workload's blocks
+    (ORACLE_SAMPLE_BLOCKS); returns (ms per full step extrapolated by block
+    count, description, threads)."""
     import numpy as np
     from oracle import step as ostep, roots
     from matrix_inverse_roots_stack_b200 import workloads as wl
@@ -219,16 +225,15 @@ def oracle_sample(spec, args, budget_s=15.0, seed=0):
                        solver={"ndb": "ndb", "cheb": "cheb"}.get(args.solver, "cn"), cheb_degree=args.degree,
                        cn_iters=args.cn_iters)
     V0 = wl.pi_start_vectors(B, 32, seed=0).astype(np.float64)
+    target = ORACLE_SAMPLE_BLOCKS[args.workload]
     if spec["shapes"] is None:  # standalone roots: time per matrix
         nmat = spec.get("n", 256)
-        A, _, _ = wl.spd_stack_decaying(n=min(4, nmat), b=B, seed=seed)
+        A, _, _ = wl.spd_stack_decaying(n=min(target, nmat), b=B, seed=seed)
         t0 = time.perf_counter()
         done = 0
         for i in range(A.shape[0]):
             ostep.inverse_fourth_root(A[i].astype(np.float64), V0, hp)  # power iteration + the solver
             done += 1
-            if time.perf_counter() - t0 > budget_s:
-                break
         dt = time.perf_counter() - t0
         return (dt / done * nmat * 1e3, f"{done} of {nmat} matrices ({B}x{B}), extrapolated x{nmat / done:.1f}",
                 threads)
@@ -244,7 +249,7 @@ def oracle_sample(spec, args, budget_s=15.0, seed=0):
         ostep.shampoo_step([th], [G], state, hp, V0)
         done_blocks += len(block_sizes([(r, c)], B))
         used.append(f"{r}x{c}")
-        if time.perf_counter() - t0 > budget_s:
+        if done_blocks >= target:
             break
     dt = time.perf_counter() - t0
     frac = total_blocks / done_blocks
@@ -280,7 +285,7 @@ def run_reference(args, spec, rank):
         return
     per_step = []
     for i in range(args.warmup + args.steps):
-        ms, sample, threads = oracle_sample(spec, args, budget_s=8.0)
+        ms, sample, threads = oracle_sample(spec, args)
         if i >= args.warmup:
             per_step.append(ms)
     ms = statistics.median(per_step)
@@ -387,6 +392,7 @@ def main():
 
         def step_fn():
             live["sharded"].step()
+        eager_fn = step_fn
 
         def e2e_fn(host_g, host_p):
             # the same step through the C ABI with host buffers: upload the
@@ -431,9 +437,9 @@ def main():
         step_fn = graph.replay
         ctx_info["cuda_graph"] = "timed steps replay one captured root call; per-launch figures from eager calls"
 
-    # ---------------- timed region
+    # ---------------- timed region (no per-launch events: profiling off)
     bd.profile_reset()
-    bd.profile_enable(graph is None)
+    bd.profile_enable(False)
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
@@ -447,21 +453,34 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clock_info = clocks.stop()
-    bd.profile_enable(False)
-    prof = bd.profile_read()
-    if graph is not None:
-        bd.profile_reset()
-        bd.profile_enable(True)
-        for _ in range(args.steps):
-            eager_fn()
-        torch.cuda.synchronize()
-        bd.profile_enable(False)
-        prof = bd.profile_read()
+    launches = bd.profile_read()["launches"]  # kernels launched in the timed steps (eager calls)
     ms = t_start.elapsed_time(t_stop) / args.steps
     if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
+
+    # ---------------- instrumented pass: the next steps again, with a CUDA
+    # event pair around every GEMM launch and stage (per-launch roofline and
+    # stage times; its step time is reported beside the headline)
+    prof_steps = min(args.steps, 3)
+    bd.profile_reset()
+    bd.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    p_start = torch.cuda.Event(enable_timing=True)
+    p_stop = torch.cuda.Event(enable_timing=True)
+    p_start.record(stream)
+    for _ in range(prof_steps):
+        eager_fn()
+    p_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    bd.profile_enable(False)
+    prof = bd.profile_read()
+    prof_ms = p_start.elapsed_time(p_stop) / prof_steps
+    if graph is not None:
+        launches = prof["launches"] * args.steps // prof_steps  # a replay launches what an eager call does
 
     # ---------------- end to end through host buffers
     e2e = None
@@ -524,27 +543,41 @@ def main():
             dist.destroy_process_group()
         return 0
 
-    # ---------------- roofline of the dominant kernel (the split-fp16 GEMM)
+    # ---------------- roofline of the dominant kernel (a split-fp16 GEMM)
     peaks, peak_kind = load_peaks()
-    g_ms, g_n, g_flops = prof["gemm"]
     tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    avg_ms = g_ms / max(g_n, 1)
-    # executed fp16 MMA flops as the library records them (3 per useful product, 1 in fp16 mode)
-    achieved = (g_flops / max(g_n, 1)) / (avg_ms * 1e-3) / 1e12 if g_n else None
-    bpf = GEMM_DRAM_BYTES_PER_FLOP.get((B, args.solver))
+    kernels = {"gemm_wide_kernel": prof["gemm_wide"], "gemm_split_kernel": prof["gemm"]}
+
+    def kernel_line(ms_, n_, fl_):
+        avg = ms_ / max(n_, 1)
+        # executed fp16 MMA flops as the library records them (3 per useful product, 1 in fp16 mode)
+        ach = (fl_ / max(n_, 1)) / (avg * 1e-3) / 1e12 if n_ else None
+        return avg, ach
+
+    name = max(kernels, key=lambda k: kernels[k][0])
+    g_ms, g_n, g_flops = kernels[name]
+    avg_ms, achieved = kernel_line(g_ms, g_n, g_flops)
+    # DRAM bytes per executed flop were captured on the 128 x 128 kernel
+    bpf = GEMM_DRAM_BYTES_PER_FLOP.get((B, args.solver)) if name == "gemm_split_kernel" else None
     traffic = round(bpf * g_flops / g_n) if (bpf and g_n) else None
-    roofline = {"kernel": "gemm_split_kernel", "bound": "tensor",
+    roofline = {"kernel": name, "bound": "tensor",
                 "achieved": round(achieved, 1) if achieved else None, "peak": tensor_peak,
                 "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4) if achieved else None,
                 "traffic": traffic, "traffic_unit": "bytes per launch (ncu DRAM read+write, scaled by executed flops)"
                 if traffic else None, "peak_kind": f"{peak_kind} bf16/fp16 dense, sustained",
                 "launches": g_n, "avg_launch_ms": round(avg_ms, 4),
-                "share_of_step": round(g_ms / (ms * args.steps), 4)}
+                "share_of_step": round(g_ms / (prof_ms * prof_steps), 4),
+                "measured_in": f"instrumented pass of {prof_steps} steps after the timed ones "
+                               f"({round(prof_ms, 3)} ms per step with the events)",
+                "gemm_kernels": {k: {"launches": v[1], "ms": round(v[0] / prof_steps, 3),
+                                     "tflops_executed": round(kernel_line(*v)[1], 1) if v[1] else None}
+                                 for k, v in kernels.items()},
+                "wide_kernel_regs": prof.get("wide_regs")}
 
     # ---------------- root-stage TFLOP/s vs dense TF32 peak
     s_ms = prof["solver"][0] + prof["power_iteration"][0]
     if graph is not None:
-        s_ms = ms * args.steps  # the standalone step is the root stage
+        s_ms = ms * prof_steps  # the standalone step is the root stage (graph replays, no events)
     if args.solver == "ndb":
         gemms = 2 * (3 * iters - 3)            # both stages, first-iteration and last-iteration savings
     elif args.solver in ("cn", "cn16"):
@@ -554,24 +587,26 @@ def main():
     padded = 2.0 * B ** 3 * gemms * n_factors
     unpadded = sum(2.0 * b ** 3 * gemms for b in factor_sizes)
     tf32_peak = tensor_peak / 2.0
-    # timed steps are W+1 .. W+K; roots are computed on steps with (t-1) % f == 0
+    # instrumented steps are W+K+1 .. W+K+P; roots are computed on steps with (t-1) % f == 0
     every = max(1, args.root_every) if spec["shapes"] is not None else 1
-    root_steps = sum(1 for t in range(args.warmup + 1, args.warmup + args.steps + 1) if (t - 1) % every == 0)
+    t0_step = args.warmup + args.steps
+    root_steps = sum(1 for t in range(t0_step + 1, t0_step + prof_steps + 1) if (t - 1) % every == 0)
     inverse_root = None
     if root_steps and s_ms > 0:
         root_s = s_ms * 1e-3 / root_steps
-        inverse_root = {"ms_per_root_step": round(root_s * 1e3, 3), "root_steps_timed": root_steps,
+        inverse_root = {"ms_per_root_step": round(root_s * 1e3, 3), "root_steps_profiled": root_steps,
                         "tflops": round(padded / root_s / 1e12, 1),
                         "tflops_unpadded": round(unpadded / root_s / 1e12, 1),
                         "tf32_peak_tflops": tf32_peak,
                         "frac_of_tf32_peak": round(padded / root_s / 1e12 / tf32_peak, 4),
                         "frac_of_tf32_peak_unpadded": round(unpadded / root_s / 1e12 / tf32_peak, 4),
                         "peak_kind": f"{peak_kind}: bf16 sustained x 0.5 (nominal TF32/BF16 ratio)"}
-    stages = {k: round(v[0] / args.steps, 3) for k, v in prof.items() if isinstance(v, tuple) and k != "gemm"}
+    stages = {k: round(v[0] / prof_steps, 3) for k, v in prof.items()
+              if isinstance(v, tuple) and k not in ("gemm", "gemm_wide")}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        c_ms, sample, threads = oracle_sample(spec, args, budget_s=15.0)
+        c_ms, sample, threads = oracle_sample(spec, args)
         cpu = {"value": round(c_ms, 1), "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample}
 
     line = {"metric": "Shampoo optimizer step ms", "value": round(ms, 3), "unit": "ms", "n_gpus": world,
@@ -582,7 +617,7 @@ def main():
             "data": "synthetic",
             "config": arm_config(args, spec, world), "state": ctx_info,
             "roofline": roofline, "inverse_root": inverse_root, "stage_ms": stages,
-            "gpu_launches": prof["launches"], "clocks": clock_info, "e2e": e2e, "cpu_baseline": cpu}
+            "gpu_launches": launches, "clocks": clock_info, "e2e": e2e, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -219,7 +219,7 @@ def read_static_status(stream=None):
     return rc, flags.value
 
 
-PROFILE_STAGES = ("gemm", "accumulate", "power_iteration", "solver", "precondition", "adam_update")
+PROFILE_STAGES = ("gemm", "accumulate", "power_iteration", "solver", "precondition", "adam_update", "gemm_wide")
 
 
 def profile_enable(on=True):
@@ -232,11 +232,13 @@ def profile_reset():
 
 def profile_read():
     """Return {stage: (ms, count, flops)}, plus "launches" and "dropped"."""
-    buf = (ctypes.c_double * 20)()
-    _check(load().shampoo_profile_read(buf, 20), "shampoo_profile_read")
+    n = 3 * len(PROFILE_STAGES) + 3
+    buf = (ctypes.c_double * n)()
+    _check(load().shampoo_profile_read(buf, n), "shampoo_profile_read")
     out = {s: (buf[3 * i], int(buf[3 * i + 1]), buf[3 * i + 2]) for i, s in enumerate(PROFILE_STAGES)}
-    out["launches"] = int(buf[18])
-    out["dropped"] = int(buf[19])
+    out["launches"] = int(buf[n - 3])
+    out["dropped"] = int(buf[n - 2])
+    out["wide_regs"] = int(buf[n - 1])
     return out
 
 

@@ -207,6 +207,7 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
         o.out_split = X_split;
         o.out_f32 = X_f32;
         o.scale = xscale;
+        o.split_norm = 1;
         DASH_TRY(dash::launch_gemm_split(ob, g, st));
       }
     }
@@ -258,6 +259,7 @@ int run_cheb_chunk(const float* F, int n, int B, float eps, const int* fsize, co
     o.alpha = 1.0f;
     o.gamma = static_cast<float>(0.5 * c[0] - c[2]);
     o.scale = xscale;
+    o.split_norm = 1;
     o.out_f32 = X_f32;
     o.out_split = X_split;
     DASH_TRY(dash::launch_gemm_split(ob, g, st));
@@ -296,6 +298,7 @@ int run_cheb_chunk(const float* F, int n, int B, float eps, const int* fsize, co
     o.cin_i.base = slot(2);
     o.gamma = static_cast<float>(0.5 * c[0]);
     o.scale = xscale;
+    o.split_norm = 1;
     o.out_f32 = X_f32;
     o.out_split = X_split;
     DASH_TRY(dash::launch_gemm_split(ob, g, st));
@@ -377,6 +380,7 @@ int run_cn_chunk(const float* F, int n, int B, float eps, const int* fsize, cons
         o.out_split = X_split;
         o.out_f32 = X_f32;
         o.scale = xscale;
+        o.split_norm = 1;
       } else {
         o.out_split = Xb[xc ^ 1];
       }
@@ -475,7 +479,7 @@ struct shampoo_ctx {
   int n_blocks = 0, n_factors = 0;
   RootLayout roots{};
   size_t off_gs = 0, off_roots = 0, off_u = 0, off_pn = 0, off_un = 0, off_blocks = 0, off_params = 0,
-         off_prefix = 0, off_fsize = 0, off_step = 0, total = 0;
+         off_prefix = 0, off_fsize = 0, off_step = 0, off_gmax = 0, off_fscale2 = 0, off_bscale = 0, off_uscale = 0, total = 0;
   const void* tables_ws = nullptr;
   const void* roots_ws = nullptr;  // workspace holding the roots of the last root step
   const void* step_ws = nullptr;   // workspace whose step counter an explicit step has set
@@ -603,6 +607,10 @@ int shampoo_init_blocks(shampoo_ctx** out, const shampoo_param* params, int n_pa
   c->off_prefix = b.take(sizeof(long long) * (n_params + 1));
   c->off_fsize = b.take(sizeof(int) * c->n_factors);
   c->off_step = b.take(4 * sizeof(int));  // step counter and the Adam bias corrections
+  c->off_gmax = b.take(sizeof(unsigned) * c->n_blocks);  // gradient scaling: max |G_k| bits,
+  c->off_fscale2 = b.take(sizeof(float) * c->n_factors);  // 2^(2 e_k) per factor,
+  c->off_bscale = b.take(sizeof(float) * c->n_blocks);    // 2^(e_k) per block
+  c->off_uscale = b.take(sizeof(float) * c->n_blocks);    // split roots: 2^(e_L + e_R) per block
   c->total = b.off;
   *workspace_bytes = c->total;
   *out = c;
@@ -655,15 +663,22 @@ int shampoo_accumulate(shampoo_ctx* ctx, float* factors, void* ws_v, size_t ws_b
   DASH_TRY(cudaMemsetAsync(status, 0, sizeof(unsigned), st));
   const int B = ctx->B;
   __half* Gs = split_at(ws, ctx->off_gs, 0, B);
+  unsigned* gmax = reinterpret_cast<unsigned*>(ws + ctx->off_gmax);
+  float* fscale2 = reinterpret_cast<float*>(ws + ctx->off_fscale2);
   const int aslot = dash::prof_begin(dash::kProfAccumulate, st);
+  DASH_TRY(cudaMemsetAsync(gmax, 0, sizeof(unsigned) * ctx->n_blocks, st));
+  // each block is gathered scaled by 2^-e (its entries then lie in (-1, 1), the
+  // split-fp16 operand range), and the products undo it exactly
   dash::launch_gather(reinterpret_cast<const BlockDesc*>(ws + ctx->off_blocks),
-                      reinterpret_cast<const ParamDev*>(ws + ctx->off_params), ctx->n_blocks, B, Gs, st);
+                      reinterpret_cast<const ParamDev*>(ws + ctx->off_params), ctx->n_blocks, B, gmax, fscale2,
+                      reinterpret_cast<float*>(ws + ctx->off_bscale), Gs, st);
   DASH_LAUNCHED();
   // L <- beta L + (1-beta) G G^T ; R <- beta R + (1-beta) G^T G   (factor f uses Gs[f] twice)
   GemmArgs g = gemm_args(B, 1, status);
   dash::GemmOp& o = g.op[0];
   o.nprob = ctx->n_factors;
   o.alpha = 1.0f - ctx->hp.beta;
+  o.acc_scale = fscale2;  // 2^(2e): (2^-e G)(2^-e G)^T = 2^-2e G G^T
   o.beta = ctx->hp.beta;
   o.cin_f32 = factors;
   o.out_f32 = factors;
@@ -724,13 +739,20 @@ int shampoo_precondition_step(shampoo_ctx* ctx, const float* factors, const floa
     dash::OpBuffers ob[2] = {{Gs, nf, roots, nf}, {Gs, nf, roots, nf}};
     DASH_TRY(dash::launch_gemm_split(ob, g, st));
   }
-  {  // U_k = X_L T1_k, scattered into parameter layout with ||U_k||^2   (A = X_L, B = T1_k)
+  {  // U_k = X_L T1_k, scattered into parameter layout with ||U_k||^2   (A = X_L, B = T1_k);
+     // T1 was formed from the gathered 2^-e G and both split roots were stored
+     // without their scales' powers of two, so U_k is multiplied back by them
+    float* uscale = reinterpret_cast<float*>(ws + ctx->off_uscale);
+    dash::launch_root_pair_scale(reinterpret_cast<const float*>(ws + ctx->roots.xscale), nb, uscale, st);
+    DASH_LAUNCHED();
     GemmArgs g = gemm_args(B, 0, status);
     dash::GemmOp& o = g.op[0];
     o.nprob = nb;
     o.a.stride = 2;
     o.b_mn = 1;
     o.alpha = 1.0f;
+    o.acc_scale = uscale;
+    o.scale = reinterpret_cast<const float*>(ws + ctx->off_bscale);
     o.blocks = reinterpret_cast<const BlockDesc*>(ws + ctx->off_blocks);
     o.u_out = U;
     o.unorm = un;

@@ -25,6 +25,7 @@
 // epilogue (scales, Cin, identity shift) and store the parked tile: the
 // ring keeps draining while a tile is written out.
 #include "gemm.cuh"
+#include "gemm_common.cuh"
 #include "launch_util.cuh"
 #include "profile.cuh"
 #include "ptx.cuh"
@@ -57,10 +58,6 @@ struct Bars {
   int abort;
 };
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + static_cast<int>(sizeof(Bars)) + 64;
-
-__device__ __forceinline__ int at(const Idx& i, int p) {
-  return i.base + (i.stride > 0 ? i.stride : 1) * (i.mod > 0 ? p % i.mod : p);
-}
 
 // Tile t of a problem -> (tile row, tile column).  sym: upper triangle of
 // the nt x nt square tile grid only, enumerated row by row.
@@ -97,84 +94,6 @@ __device__ __forceinline__ void decode(const GemmArgs& args, int tpp, int ntn, l
   const long long u = op ? t - n0 : t;
   p = static_cast<int>(u / tpp);
   tile_coords(static_cast<int>(u % tpp), ntn, args.sym, ti, tj);
-}
-
-__device__ __forceinline__ void fail_timeout(volatile int* abort_flag, unsigned* status) {
-  *abort_flag = 1;
-  if (status) atomicOr(status, kStatusTimeout);
-}
-
-// Descriptor of an MN-major operand tile: 64 K-rows of 128 bytes per
-// 64-column box, boxes 8 KB apart (leading byte offset), 8-row swizzle atoms
-// of 1024 bytes (stride byte offset), 128-byte swizzle.
-__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(8192u >> 4) << 16;
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
-  return d;
-}
-
-__device__ __forceinline__ void store_split16(__half* base, size_t BB, size_t idx, const float* v, bool& bad) {
-  __half hi[16], lo[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    split_f16(v[j], hi[j], lo[j]);
-    bad |= (__hisinf(hi[j]) != 0);
-  }
-  uint4* dh = reinterpret_cast<uint4*>(base + idx);
-  uint4* dl = reinterpret_cast<uint4*>(base + BB + idx);
-  dh[0] = *reinterpret_cast<const uint4*>(&hi[0]);
-  dh[1] = *reinterpret_cast<const uint4*>(&hi[8]);
-  dl[0] = *reinterpret_cast<const uint4*>(&lo[0]);
-  dl[1] = *reinterpret_cast<const uint4*>(&lo[8]);
-}
-
-// out(col0 + j, row) = v[j]: for a fixed j the 32 lanes (consecutive rows)
-// write consecutive addresses.
-__device__ __forceinline__ void store_split16_t(__half* base, size_t B, size_t BB, int row, int col0, const float* v,
-                                                bool& bad) {
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    __half h, l;
-    split_f16(v[j], h, l);
-    bad |= (__hisinf(h) != 0);
-    base[(col0 + j) * B + row] = h;
-    base[BB + (col0 + j) * B + row] = l;
-  }
-}
-
-// Raw 16-element chunk of a split row (hi and lo planes, 32 bytes each).
-struct SplitChunk {
-  uint4 h[2], l[2];
-};
-
-__device__ __forceinline__ SplitChunk ld_chunk(const __half* base, size_t BB, size_t idx) {
-  SplitChunk c;
-  const uint4* h4 = reinterpret_cast<const uint4*>(base + idx);
-  const uint4* l4 = reinterpret_cast<const uint4*>(base + BB + idx);
-  c.h[0] = h4[0];
-  c.h[1] = h4[1];
-  c.l[0] = l4[0];
-  c.l[1] = l4[1];
-  return c;
-}
-
-__device__ __forceinline__ void join_chunk(const SplitChunk& c, float* out) {
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const __half2* ah = reinterpret_cast<const __half2*>(&c.h[q]);
-    const __half2* bh = reinterpret_cast<const __half2*>(&c.l[q]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 x = __half22float2(ah[e]);
-      const float2 y = __half22float2(bh[e]);
-      out[q * 8 + 2 * e] = x.x + y.x * kLoUnscale;
-      out[q * 8 + 2 * e + 1] = x.y + y.y * kLoUnscale;
-    }
-  }
 }
 
 // kSingle: one pass of hi*hi only (fp16 operands, fp32 accumulation); the lo
@@ -233,12 +152,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         int op, p, ti, tj;
         decode(args, tpp, nt, t, op, p, ti, tj);
         const GemmOp& g = args.op[op];
-        const int am = at(g.a, p), bm = at(g.b, p);
+        const int am = gemm_at(g.a, p), bm = gemm_at(g.b, p);
         const CUtensorMap* ta = op ? &tmA1 : &tmA0;
         const CUtensorMap* tb = op ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb, ++sc) {
           if (!mbar_wait(&bars->empty[s], epar, abort_flag)) {  // fresh barriers pass on parity 1
-            fail_timeout(abort_flag, args.status);
+            gemm_fail_timeout(abort_flag, args.status);
             stop = true;
             break;
           }
@@ -329,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) fail_timeout(abort_flag, args.status);
+      if (!ok) gemm_fail_timeout(abort_flag, args.status);
       // all issued MMAs must retire before tensor memory is released
       mma_commit(&bars->drain);
       volatile int never = 0;
@@ -378,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ppar ^= 1u;
       }
       if (!ok) {
-        if (threadIdx.x == kAccWarp0 * 32) fail_timeout(abort_flag, args.status);
+        if (threadIdx.x == kAccWarp0 * 32) gemm_fail_timeout(abort_flag, args.status);
         break;
       }
       tc_fence_after();
@@ -402,28 +321,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const GemmOp& g = args.op[op];
       const int row = ti * kTile + quad * 32 + lane;
       const int cbase = tj * kTile;
-      const float s = g.scale ? g.scale[at(g.scale_i, p)] : 1.0f;
-      const __half* cin = g.cin_split ? g.cin_split + static_cast<size_t>(at(g.cin_i, p)) * 2 * BB : nullptr;
-      const float* cinf = g.cin_f32 ? g.cin_f32 + static_cast<size_t>(at(g.cinf_i, p)) * BB : nullptr;
-      __half* os = g.out_split ? g.out_split + static_cast<size_t>(at(g.out_i, p)) * 2 * BB : nullptr;
-      float* of = g.out_f32 ? g.out_f32 + static_cast<size_t>(at(g.outf_i, p)) * BB : nullptr;
       const bool mirror = args.sym && (ti != tj);
-      BlockDesc bd;
-      if (g.blocks) bd = g.blocks[p];
-      SplitChunk nxt;  // Cin is loaded one chunk ahead, the first before the wait
-      if (cin) nxt = ld_chunk(cin, BB, row * B + cbase);
+      GemmEpilogue ep;
+      ep.init(g, p, B, BB);
+      GemmEpilogue::CinRaw nxt;  // Cin is loaded one chunk ahead, the first before the wait
+      if (ep.has_cin()) nxt = ep.load_cin(B, BB, row, cbase);
       if (!mbar_wait_sleep(&bars->park_full, ppar, abort_flag)) {
-        if (threadIdx.x == kOutWarp0 * 32) fail_timeout(abort_flag, args.status);
+        if (threadIdx.x == kOutWarp0 * 32) gemm_fail_timeout(abort_flag, args.status);
         break;
       }
       ppar ^= 1u;
       tc_fence_after();
-      bool bad = false;
-      float sumsq = 0.0f;
 #pragma unroll 1
       for (int c = 0; c < kTile / 16; ++c) {
         const int col0 = cbase + c * 16;
-        float v[16];
+        float v[16], cj[16];
         tmem_ld_32x32b_x16(tbase + lane_off + kColPark + 16 * c, reinterpret_cast<uint32_t*>(v));
         tmem_ld_wait();
         if (c + 1 == kTile / 16) {  // the park buffer is free for the next tile
@@ -431,70 +343,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->park_empty);
         }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] *= g.alpha;
-        if (cin) {
-          const SplitChunk cur = nxt;
-          if (c + 1 < kTile / 16) nxt = ld_chunk(cin, BB, row * B + col0 + 16);
-          float cj[16];
-          join_chunk(cur, cj);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] += g.beta * cj[j];
+        if (ep.has_cin()) {
+          const GemmEpilogue::CinRaw cur = nxt;
+          if (c + 1 < kTile / 16) nxt = ep.load_cin(B, BB, row, col0 + 16);
+          ep.join_cin(cur, cj);
         }
-        if (cinf) {
-          const float4* c4 = reinterpret_cast<const float4*>(cinf + row * B + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 cq = c4[q];
-            v[4 * q] += g.beta * cq.x;
-            v[4 * q + 1] += g.beta * cq.y;
-            v[4 * q + 2] += g.beta * cq.z;
-            v[4 * q + 3] += g.beta * cq.w;
-          }
-        }
-        if (g.gamma != 0.0f) {
-          const int d = row - col0;
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j == d) v[j] += g.gamma;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] *= s;
-          bad |= !isfinite(v[j]);
-        }
-        if (g.blocks) {
-          if (row < bd.br) {
-            float* dst = g.u_out + bd.off + static_cast<long long>(bd.r0 + row) * bd.pitch + bd.c0 + col0;
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (col0 + j < bd.bc) {
-                dst[j] = v[j];
-                sumsq += v[j] * v[j];
-              }
-          }
-          continue;
-        }
-        if (os) {
-          store_split16(os, BB, row * B + col0, v, bad);
-          if (mirror) store_split16_t(os, B, BB, row, col0, v, bad);
-        }
-        if (of) {
-          float4* d4 = reinterpret_cast<float4*>(of + row * B + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          if (mirror) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) of[(col0 + j) * B + row] = v[j];
-          }
-        }
+        ep.chunk(g, B, BB, row, col0, v, cj, mirror);
       }
-      if (bad) atomicOr(args.status, kStatusNonFinite);
-      if (g.blocks) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-        if (lane == 0 && sumsq != 0.0f) atomicAdd(&g.unorm[p], sumsq);
-      }
+      ep.finish(g, p, args.status);
     }
   }
 
@@ -508,14 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 std::atomic<int> g_load_fault{0};
 
-int sm_count() {
+}  // namespace
+
+int gemm_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
   return n;
 }
-
-}  // namespace
 
 cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaStream_t stream) {
   if (args.nops < 1 || args.nops > 2) return cudaErrorInvalidValue;
@@ -525,14 +381,16 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   GemmArgs a = args;
   if (a.nops == 1) a.op[1] = a.op[0], a.op[1].nprob = 0;
   if (g_load_fault.exchange(0) != 0) a.skip_loads = 1;
+  const bool wide = gemm_wide_supported(a);
   CUtensorMap maps[4];
   for (int o = 0; o < 2; ++o) {
     const OpBuffers& b = bufs[o < a.nops ? o : 0];
     cudaError_t e = encode_split_stack_map(&maps[2 * o], b.a, a.B, b.a_nmat, kTile);
     if (e != cudaSuccess) return e;
-    e = encode_split_stack_map(&maps[2 * o + 1], b.b, a.B, b.b_nmat, a.op[o].b_mn ? 64 : kTile);
+    e = encode_split_stack_map(&maps[2 * o + 1], b.b, a.B, b.b_nmat, a.op[o].b_mn ? 64 : (wide ? 256 : kTile));
     if (e != cudaSuccess) return e;
   }
+  if (wide) return launch_gemm_wide(maps, a, nprob, stream);
   void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmArgs,
                const long long) = a.single_pass ? gemm_split_kernel<true> : gemm_split_kernel<false>;
   static std::atomic<unsigned long long> attr_set[2];
@@ -541,7 +399,7 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   const long long nt = a.B / kTile;
   const long long tpp = a.sym ? nt * (nt + 1) / 2 : nt * nt;
   const long long total = tpp * nprob;
-  const long long sms = sm_count();
+  const long long sms = gemm_sm_count();
   const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
   // executed tensor-core flops: each computed 128 x 128 tile is one
   // 2*128*128*B product, done as three fp16 products (one in single-pass mode)

@@ -9,8 +9,9 @@
 // fp32 registers, which gives about fp32 accuracy at the fp16 tensor-core rate.
 //
 // Problem p computes
-//     out_p = s_p * (alpha * A_p op(B_p) + beta * Cin_p + gamma * I)
-// where A_p is a row-major matrix of the A stack (read K-major) and op(B_p)
+//     out_p = s_p * (alpha * a_p * A_p op(B_p) + beta * Cin_p + gamma * I)
+// (s_p, a_p optional per-problem scalars) where A_p is a row-major matrix of
+// the A stack (read K-major) and op(B_p)
 // is B_p (b_mn = 1: the stored row-major B is read MN-major, giving A B) or
 // B_p^T (b_mn = 0: read K-major, giving A B^T).  A launch carries one or two
 // "ops" (groups of problems) with their own operand stacks and epilogues.
@@ -48,12 +49,15 @@ struct GemmOp {
   float alpha, beta, gamma;
   const float* scale;        // per-problem multiplier s_p (nullptr: 1)
   Idx scale_i;
+  const float* acc_scale;    // per-problem multiplier of alpha alone (nullptr: 1)
+  Idx accs_i;
   const __half* cin_split;   // split Cin stack (nullptr: none)
   Idx cin_i;
   const float* cin_f32;      // fp32 Cin stack (nullptr: none)
   Idx cinf_i;
   __half* out_split;         // split output (+ mirror if sym)
   Idx out_i;
+  int split_norm;            // 1: the split output is out_p * 2^-e with 2^(e-1) <= s_p < 2^e
   float* out_f32;            // fp32 output (+ mirror if sym)
   Idx outf_i;
   const BlockDesc* blocks;   // non-null: scatter out_p into u_out (parameter layout)

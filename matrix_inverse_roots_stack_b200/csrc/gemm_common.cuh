@@ -1,0 +1,243 @@
+// Pieces shared by the two split-fp16 GEMM kernels (gemm.cu: 128 x 128 tiles
+// with a parked output stage; gemm_wide.cu: 128 x 256 tiles written out by
+// the accumulator warps): problem indexing, the MN-major operand descriptor,
+// the split-fp16 load/store helpers and the epilogue of one output row
+// segment, out = s_p * (alpha * a_p * acc + beta * Cin + gamma * I).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace dash {
+
+__device__ __forceinline__ int gemm_at(const Idx& i, int p) {
+  return i.base + (i.stride > 0 ? i.stride : 1) * (i.mod > 0 ? p % i.mod : p);
+}
+
+__device__ __forceinline__ void gemm_fail_timeout(volatile int* abort_flag, unsigned* status) {
+  *abort_flag = 1;
+  if (status) atomicOr(status, kStatusTimeout);
+}
+
+// Descriptor of an MN-major operand tile: 64 K-rows of 128 bytes per
+// 64-column box, boxes 8 KB apart (leading byte offset), 8-row swizzle atoms
+// of 1024 bytes (stride byte offset), 128-byte swizzle.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(8192u >> 4) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void store_split16(__half* base, size_t BB, size_t idx, const float* v, bool& bad) {
+  __half hi[16], lo[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    split_f16(v[j], hi[j], lo[j]);
+    bad |= (__hisinf(hi[j]) != 0);
+  }
+  uint4* dh = reinterpret_cast<uint4*>(base + idx);
+  uint4* dl = reinterpret_cast<uint4*>(base + BB + idx);
+  dh[0] = *reinterpret_cast<const uint4*>(&hi[0]);
+  dh[1] = *reinterpret_cast<const uint4*>(&hi[8]);
+  dl[0] = *reinterpret_cast<const uint4*>(&lo[0]);
+  dl[1] = *reinterpret_cast<const uint4*>(&lo[8]);
+}
+
+// out(col0 + j, row) = v[j]: for a fixed j the 32 lanes (consecutive rows)
+// write consecutive addresses.
+__device__ __forceinline__ void store_split16_t(__half* base, size_t B, size_t BB, int row, int col0, const float* v,
+                                                bool& bad) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    __half h, l;
+    split_f16(v[j], h, l);
+    bad |= (__hisinf(h) != 0);
+    base[(col0 + j) * B + row] = h;
+    base[BB + (col0 + j) * B + row] = l;
+  }
+}
+
+// Raw 16-element chunk of a split row (hi and lo planes, 32 bytes each).
+struct SplitChunk {
+  uint4 h[2], l[2];
+};
+
+__device__ __forceinline__ SplitChunk ld_chunk(const __half* base, size_t BB, size_t idx) {
+  SplitChunk c;
+  const uint4* h4 = reinterpret_cast<const uint4*>(base + idx);
+  const uint4* l4 = reinterpret_cast<const uint4*>(base + BB + idx);
+  c.h[0] = h4[0];
+  c.h[1] = h4[1];
+  c.l[0] = l4[0];
+  c.l[1] = l4[1];
+  return c;
+}
+
+__device__ __forceinline__ void join_chunk(const SplitChunk& c, float* out) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const __half2* ah = reinterpret_cast<const __half2*>(&c.h[q]);
+    const __half2* bh = reinterpret_cast<const __half2*>(&c.l[q]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __half22float2(ah[e]);
+      const float2 y = __half22float2(bh[e]);
+      out[q * 8 + 2 * e] = x.x + y.x * kLoUnscale;
+      out[q * 8 + 2 * e + 1] = x.y + y.y * kLoUnscale;
+    }
+  }
+}
+
+// Epilogue of one problem's output for a run of 16-column chunks of one row:
+// v = s_p * (alpha * a_p * acc + beta * Cin + gamma * I), written as split
+// fp16 (times 2^-e when split_norm is set, 2^(e-1) <= s_p < 2^e) and/or fp32
+// (mirrored for symmetric launches), or scattered into parameter layout with
+// its sum of squares.
+struct GemmEpilogue {
+  float s, alpha, beta, gamma, ss;
+  const __half* cin;
+  const float* cinf;
+  __half* os;
+  float* of;
+  bool scatter;
+  BlockDesc bd;
+  float sumsq;
+  bool bad;
+
+  __device__ __forceinline__ void init(const GemmOp& g, int p, size_t B, size_t BB) {
+    (void)B;
+    s = g.scale ? g.scale[gemm_at(g.scale_i, p)] : 1.0f;
+    ss = 1.0f;  // split outputs of root stacks carry s_p's power of two back out (fp16 range)
+    if (g.split_norm && isfinite(s) && s != 0.0f) {
+      int e;
+      frexpf(s, &e);
+      ss = ldexpf(1.0f, -e);
+    }
+    alpha = g.acc_scale ? g.alpha * g.acc_scale[gemm_at(g.accs_i, p)] : g.alpha;
+    beta = g.beta;
+    gamma = g.gamma;
+    cin = g.cin_split ? g.cin_split + static_cast<size_t>(gemm_at(g.cin_i, p)) * 2 * BB : nullptr;
+    cinf = g.cin_f32 ? g.cin_f32 + static_cast<size_t>(gemm_at(g.cinf_i, p)) * BB : nullptr;
+    os = g.out_split ? g.out_split + static_cast<size_t>(gemm_at(g.out_i, p)) * 2 * BB : nullptr;
+    of = g.out_f32 ? g.out_f32 + static_cast<size_t>(gemm_at(g.outf_i, p)) * BB : nullptr;
+    scatter = g.blocks != nullptr;
+    if (scatter) bd = g.blocks[p];
+    sumsq = 0.0f;
+    bad = false;
+  }
+
+  // Raw Cin of one 16-column chunk (64 bytes: split hi and lo planes, or
+  // fp32), so that several chunks can be in flight before any is used.
+  struct CinRaw {
+    uint4 q[4];
+  };
+  __device__ __forceinline__ bool has_cin() const { return cin != nullptr || cinf != nullptr; }
+  __device__ __forceinline__ CinRaw load_cin(size_t B, size_t BB, int row, int col0) const {
+    CinRaw r;
+    if (cin) {
+      const uint4* h = reinterpret_cast<const uint4*>(cin + row * B + col0);
+      const uint4* l = reinterpret_cast<const uint4*>(cin + BB + row * B + col0);
+      r.q[0] = h[0];
+      r.q[1] = h[1];
+      r.q[2] = l[0];
+      r.q[3] = l[1];
+    } else {
+      const uint4* f = reinterpret_cast<const uint4*>(cinf + row * B + col0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r.q[i] = f[i];
+    }
+    return r;
+  }
+  __device__ __forceinline__ void join_cin(const CinRaw& r, float* cj) const {
+    if (cin) {
+      SplitChunk c;
+      c.h[0] = r.q[0];
+      c.h[1] = r.q[1];
+      c.l[0] = r.q[2];
+      c.l[1] = r.q[3];
+      join_chunk(c, cj);
+    } else {
+      const float* f = reinterpret_cast<const float*>(r.q);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) cj[j] = f[j];
+    }
+  }
+
+  // One 16-column chunk; cj holds Cin's chunk in fp32 when has_cin().
+  __device__ __forceinline__ void chunk(const GemmOp& g, size_t B, size_t BB, int row, int col0, float* v,
+                                        const float* cj, bool mirror) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] *= alpha;
+    if (has_cin()) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] += beta * cj[j];
+    }
+    if (gamma != 0.0f) {
+      const int d = row - col0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j == d) v[j] += gamma;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      v[j] *= s;
+      bad |= !isfinite(v[j]);
+    }
+    if (scatter) {
+      if (row < bd.br) {
+        float* dst = g.u_out + bd.off + static_cast<long long>(bd.r0 + row) * bd.pitch + bd.c0 + col0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (col0 + j < bd.bc) {
+            dst[j] = v[j];
+            sumsq += v[j] * v[j];
+          }
+      }
+      return;
+    }
+    if (os) {
+      float w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) w[j] = v[j] * ss;
+      store_split16(os, BB, row * B + col0, w, bad);
+      if (mirror) store_split16_t(os, B, BB, row, col0, w, bad);
+    }
+    if (of) {
+      float4* d4 = reinterpret_cast<float4*>(of + row * B + col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      if (mirror) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) of[(col0 + j) * B + row] = v[j];
+      }
+    }
+  }
+
+  // Warp-collective: the non-finite flag and the scattered sum of squares.
+  __device__ __forceinline__ void finish(const GemmOp& g, int p, unsigned* status) {
+    if (bad) atomicOr(status, kStatusNonFinite);
+    if (scatter) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+      if ((threadIdx.x & 31) == 0 && sumsq != 0.0f) atomicAdd(&g.unorm[p], sumsq);
+    }
+  }
+};
+
+int gemm_sm_count();
+
+// The 128 x 256 tile kernel (gemm_wide.cu): whether it takes a launch, and
+// its launch on the four encoded operand maps (A0, B0, A1, B1; B maps with
+// 256-row boxes when K-major).
+bool gemm_wide_supported(const GemmArgs& a);
+cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long long nprob, cudaStream_t stream);
+
+}  // namespace dash

@@ -123,7 +123,26 @@ __global__ void __launch_bounds__(256) scale_split_kernel(const __half* __restri
 #pragma unroll
   for (int e = 0; e < 4; ++e) z[e] *= s;
   if (out_f32) *reinterpret_cast<float4*>(out_f32 + f * BB + idx) = make_float4(z[0], z[1], z[2], z[3]);
-  if (out_split) store_split4(out_split + 2 * f * BB, BB, idx, z);
+  if (out_split) {  // split roots carry the power of two of their scale back out (fp16 range)
+    int ex = 0;
+    if (isfinite(s) && s != 0.0f) frexpf(s, &ex);
+    const float ss = ldexpf(1.0f, -ex);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) z[e] *= ss;
+    store_split4(out_split + 2 * f * BB, BB, idx, z);
+  }
+}
+
+// uscale[k] = 2^(e_L + e_R): the powers of two that the split roots of block
+// k's factors (2k, 2k+1) were stored without, 2^(e-1) <= xscale < 2^e.
+__global__ void root_pair_scale_kernel(const float* __restrict__ xscale, int nb, float* __restrict__ uscale) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= nb) return;
+  int el = 0, er = 0;
+  const float sl = xscale[2 * k], sr = xscale[2 * k + 1];
+  if (isfinite(sl) && sl != 0.0f) frexpf(sl, &el);
+  if (isfinite(sr) && sr != 0.0f) frexpf(sr, &er);
+  uscale[k] = ldexpf(1.0f, el + er);
 }
 
 __global__ void __launch_bounds__(256) cheb_init_kernel(const float* __restrict__ F, int B, float eps,
@@ -183,9 +202,46 @@ __global__ void __launch_bounds__(256) cn_init_kernel(const float* __restrict__ 
 
 // ------------------------------------------------------------ gather
 
-// grid (B/32, B/32, nb), block (32, 8)
+// Largest |G| of every gradient block, as float bits (atomicMax on the bits
+// orders non-negative floats; NaN sorts above +Inf).  grid (B/32, nb), 256
+// threads: a CTA takes 32 rows of one block, a warp 4 rows.
+__global__ void __launch_bounds__(256) block_absmax_kernel(const BlockDesc* __restrict__ blocks,
+                                                           const ParamDev* __restrict__ params,
+                                                           unsigned* __restrict__ gmax) {
+  const int k = blockIdx.y;
+  const BlockDesc bd = blocks[k];
+  const float* G = params[bd.param].grad;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned m = 0u;
+  for (int i = 0; i < 4; ++i) {
+    const int r = blockIdx.x * 32 + warp * 4 + i;
+    if (r >= bd.br) break;
+    const float* row = G + static_cast<long long>(bd.r0 + r) * bd.pitch + bd.c0;
+    for (int c = lane; c < bd.bc; c += 32) m = max(m, __float_as_uint(fabsf(row[c])));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if (lane == 0 && m != 0u) atomicMax(&gmax[k], m);
+}
+
+// Power-of-two scale 2^-e of a gradient block with largest entry x:
+// 2^(e-1) <= x < 2^e, so every scaled entry lies in (-1, 1) and its fp16
+// split neither overflows nor (for entries within 2^-14 of the largest)
+// loses bits to subnormals; 1 for an all-zero or non-finite block.
+__device__ __forceinline__ int block_exponent(unsigned bits) {
+  const float x = __uint_as_float(bits);
+  if (bits == 0u || !isfinite(x)) return 0;
+  int e;
+  frexpf(x, &e);
+  return e;
+}
+
+// grid (B/32, B/32, nb), block (32, 8).  Gs[2k] = G_k 2^-e_k, Gs[2k+1] its
+// transpose; the CTA at tile (0, 0) also writes the exact factors that undo
+// the scaling: fscale2[2k] = fscale2[2k+1] = 2^(2 e_k) (for G G^T, G^T G)
+// and bscale[k] = 2^(e_k) (for X_L G X_R).
 __global__ void gather_kernel(const BlockDesc* __restrict__ blocks, const ParamDev* __restrict__ params, int B,
-                              __half* __restrict__ Gs) {
+                              const unsigned* __restrict__ gmax, float* __restrict__ fscale2,
+                              float* __restrict__ bscale, __half* __restrict__ Gs) {
   __shared__ float tile[32][33];
   const int k = blockIdx.z;
   const BlockDesc bd = blocks[k];
@@ -193,12 +249,18 @@ __global__ void gather_kernel(const BlockDesc* __restrict__ blocks, const ParamD
   const size_t BB = static_cast<size_t>(B) * B;
   __half* g0 = Gs + static_cast<size_t>(2 * k) * 2 * BB;
   __half* g1 = Gs + static_cast<size_t>(2 * k + 1) * 2 * BB;
+  const int e = block_exponent(gmax[k]);
+  const float sc = ldexpf(1.0f, -e);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
+    fscale2[2 * k] = fscale2[2 * k + 1] = ldexpf(1.0f, 2 * e);
+    bscale[k] = ldexpf(1.0f, e);
+  }
   const int tr = blockIdx.y * 32, tc = blockIdx.x * 32;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = tr + threadIdx.y + 8 * i, c = tc + threadIdx.x;
     float v = 0.0f;
-    if (r < bd.br && c < bd.bc) v = G[static_cast<long long>(bd.r0 + r) * bd.pitch + bd.c0 + c];
+    if (r < bd.br && c < bd.bc) v = sc * G[static_cast<long long>(bd.r0 + r) * bd.pitch + bd.c0 + c];
     tile[threadIdx.y + 8 * i][threadIdx.x] = v;
     __half h, l;
     split_f16(v, h, l);
@@ -415,9 +477,17 @@ void launch_cn_init(const float* F, int nf, int B, float eps, const int* fsize, 
   prof_count_launch();
 }
 
-void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int B, __half* Gs, cudaStream_t st) {
+void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int B, unsigned* gmax, float* fscale2,
+                   float* bscale, __half* Gs, cudaStream_t st) {
+  block_absmax_kernel<<<dim3(B / 32, nb), 256, 0, st>>>(blocks, params, gmax);
+  prof_count_launch();
   dim3 grid(B / 32, B / 32, nb);
-  gather_kernel<<<grid, dim3(32, 8), 0, st>>>(blocks, params, B, Gs);
+  gather_kernel<<<grid, dim3(32, 8), 0, st>>>(blocks, params, B, gmax, fscale2, bscale, Gs);
+  prof_count_launch();
+}
+
+void launch_root_pair_scale(const float* xscale, int nb, float* uscale, cudaStream_t st) {
+  root_pair_scale_kernel<<<(nb + 255) / 256, 256, 0, st>>>(xscale, nb, uscale);
   prof_count_launch();
 }
 

@@ -71,8 +71,12 @@ void launch_ndb_init(const float* F, int nf, int B, float eps, const int* fsize,
 // D0 = (I - Y)/2; Zhat1 = (I + D0)/zs.
 void launch_ndb_stage2_init(const __half* Y, int nf, int B, float zs, __half* D0, __half* Z1, cudaStream_t st);
 
-// out = xscale_f * Zhat (split in; fp32 and/or split out); used when a stage
-// has a single iteration.
+// out = xscale_f * Zhat (split in; fp32 and/or split out, the split output
+// times 2^-e with 2^(e-1) <= xscale_f < 2^e); used when a stage has a single
+// iteration.
+// uscale[k] = 2^(e_2k + e_2k+1) with 2^(e_f - 1) <= xscale_f < 2^e_f: undoes
+// the split roots' scaling in the preconditioner (nb blocks, factors 2k, 2k+1).
+void launch_root_pair_scale(const float* xscale, int nb, float* uscale, cudaStream_t st);
 void launch_scale_split(const __half* Z, int nf, int B, const float* xscale, float* out_f32, __half* out_split,
                         cudaStream_t st);
 
@@ -87,8 +91,13 @@ void launch_cheb_init(const float* F, int nf, int B, float eps, const int* fsize
 void launch_cn_init(const float* F, int nf, int B, float eps, const int* fsize, const float* lambda, __half* M0,
                     __half* X0, float* xscale, cudaStream_t st);
 
-// Gather gradient blocks into padded split matrices: Gs[2k] = G_k, Gs[2k+1] = G_k^T.
-void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int B, __half* Gs, cudaStream_t st);
+// Gather gradient blocks into padded split matrices scaled by a power of two
+// per block, 2^-e_k with 2^(e_k - 1) <= max |G_k| < 2^e_k (exact):
+// Gs[2k] = G_k 2^-e_k, Gs[2k+1] = its transpose; fscale2[2k] = fscale2[2k+1]
+// = 2^(2 e_k) and bscale[k] = 2^(e_k) undo it in the products.  gmax (nb
+// words) must be zero on entry; it receives each block's max |G| bits.
+void launch_gather(const BlockDesc* blocks, const ParamDev* params, int nb, int B, unsigned* gmax, float* fscale2,
+                   float* bscale, __half* Gs, cudaStream_t st);
 
 // factors[f] = init_scale * I.
 void launch_init_factors(float* F, int nf, int B, float init_scale, cudaStream_t st);

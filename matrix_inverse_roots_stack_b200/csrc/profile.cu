@@ -6,6 +6,8 @@
 #include "profile.cuh"
 
 namespace dash {
+
+int gemm_wide_regs();  // gemm_wide.cu
 namespace {
 
 struct Rec {
@@ -94,10 +96,10 @@ SHAMPOO_API int shampoo_profile_reset(void) {
 }
 
 SHAMPOO_API int shampoo_profile_read(double* out, int n) {
-  if (!out || n < 3 * dash::kProfStages + 2) return SHAMPOO_EINVAL;
+  if (!out || n < 3 * dash::kProfStages + 3) return SHAMPOO_EINVAL;
   dash::Prof& p = dash::prof();
   std::lock_guard<std::mutex> lk(p.mu);
-  for (int i = 0; i < 3 * dash::kProfStages + 2; ++i) out[i] = 0.0;
+  for (int i = 0; i < 3 * dash::kProfStages + 3; ++i) out[i] = 0.0;
   for (auto& r : p.recs) {
     if (cudaEventSynchronize(r.stop) != cudaSuccess) return SHAMPOO_ECUDA;
     float ms = 0.0f;
@@ -108,6 +110,7 @@ SHAMPOO_API int shampoo_profile_read(double* out, int n) {
   }
   out[3 * dash::kProfStages] = static_cast<double>(p.launches.load());
   out[3 * dash::kProfStages + 1] = static_cast<double>(p.dropped);
+  out[3 * dash::kProfStages + 2] = static_cast<double>(dash::gemm_wide_regs());
   return SHAMPOO_OK;
 }
 

@@ -11,13 +11,14 @@
 namespace dash {
 
 enum ProfStage {
-  kProfGemm = 0,         // every launch of the split-fp16 GEMM kernel
+  kProfGemm = 0,         // launches of the split-fp16 GEMM with 128 x 128 tiles (gemm.cu)
   kProfAccumulate = 1,   // gradient gather + factor EMA
   kProfPowerIter = 2,    // multi-start power iteration
   kProfSolver = 3,       // Newton-DB / Chebyshev (prologues + GEMMs)
   kProfPrecond = 4,      // U = X_L G X_R
   kProfAdam = 5,         // Adam moments, graft and update
-  kProfStages = 6
+  kProfGemmWide = 6,     // launches of the split-fp16 GEMM with 128 x 256 tiles (gemm_wide.cu)
+  kProfStages = 7
 };
 
 bool prof_on();

@@ -2,17 +2,16 @@
 sampled blocks against the float64 oracle block by block.
 
 The whole step runs on the GPU exactly as bench.py launches it; the oracle
-recomputes a few blocks (first, middle, last -- edge blocks included) from
-their gradient blocks, at the GPU's power-iteration estimates (level 2).
+recomputes the sampled blocks from their gradient blocks, at the GPU's
+power-iteration estimates (level 2).  The sample holds one block of every
+distinct block shape of the parameter set (edge blocks: 256 x 1024 rows of
+the embedding, 512-wide blocks of 5632, the 768 -> 512 + 256 and 50257 edges
+of GPT-2) and evenly spaced blocks up to at least 32 (all blocks when there
+are fewer).
 
-Tolerance on each sampled block's update (relative Frobenius error): 5e-3
-when both of its factors (with the root-time damping) have condition number
-<= 1e6, the regime the root tolerance is stated for.  First-step factors of
-these workloads reach 1e7 and more; there the error of any fp32-precision
-evaluation of the truncated iteration grows with the condition number, and
-the bound used is 5e-3 * kappa / 1e6.  The in-regime variants damp the
-factors (eps = 1e-2) so that every block satisfies kappa <= 1e6 and hold all
-of them to 5e-3.
+Tolerance on every sampled block's update (relative Frobenius error of its
+Delta theta): 5e-3, the parameter-update tolerance, whatever the factors'
+condition numbers.
 """
 
 import numpy as np
@@ -26,6 +25,7 @@ pytestmark = pytest.mark.gpu
 
 UPDATE_TOL = 5e-3
 KAPPA_REGIME = 1e6
+MIN_SAMPLE = 32
 
 
 @pytest.fixture(scope="module")
@@ -42,7 +42,26 @@ def kappa(M):
     return w[-1] / w[0]
 
 
-def run_and_check(torch, shapes, grads, B, solver="ndb", iters=14, degree=16, n_sample=6, eps=1e-6,
+def sample_blocks(table, n_sample):
+    """One block of every distinct (b_r, b_c) shape, then evenly spaced
+    blocks until n_sample (or every block)."""
+    nb = len(table)
+    picks = {}
+    for k in range(nb):
+        picks.setdefault((int(table[k][3]), int(table[k][4])), k)
+    chosen = set(picks.values())
+    for k in np.linspace(0, nb - 1, num=min(nb, n_sample)).round().astype(int):
+        if len(chosen) >= max(n_sample, len(picks)):
+            break
+        chosen.add(int(k))
+    k = 0
+    while len(chosen) < min(nb, n_sample):
+        chosen.add(k)
+        k += 1
+    return sorted(chosen)
+
+
+def run_and_check(torch, shapes, grads, B, solver="ndb", iters=14, degree=16, n_sample=MIN_SAMPLE, eps=1e-6,
                   require_regime=False):
     from matrix_inverse_roots_stack_b200 import binding as bd
     dev = grads[0].device
@@ -58,25 +77,26 @@ def run_and_check(torch, shapes, grads, B, solver="ndb", iters=14, degree=16, n_
     hp = ostep.HParams(block_size=B, solver=solver, ndb_iters1=iters, ndb_iters2=iters, cheb_degree=degree,
                        beta=f32(0.95), eps=f32(eps), init_scale=f32(1e-6), beta1=f32(0.9), beta2=f32(0.999),
                        adam_eps=f32(1e-8), lr=f32(1e-3), cheb_delta=f32(1e-3))
-    nb = len(table)
-    picks = sorted(set([0, 1, nb // 3, nb // 2, (2 * nb) // 3, nb - 1][:n_sample]))
     rows = []
-    for k in picks:
+    for k in sample_blocks(table, n_sample):
         p, r0, c0, br, bc, fl, fr = (int(x) for x in table[k])
         Gb = grads[p][r0:r0 + br, c0:c0 + bc].cpu().numpy().astype(np.float64)
         _, _, Pb = ostep.adam_direction(Gb, np.zeros_like(Gb), np.zeros_like(Gb), 1, hp)
         d_ref, _, _ = ostep.first_step_block_update(Gb, Pb, hp, lam[fl], lam[fr])
         d_gpu = params[p][r0:r0 + br, c0:c0 + bc].cpu().numpy().astype(np.float64)
         if np.linalg.norm(d_ref) == 0:
+            assert np.all(d_gpu == 0.0), k
             continue
         L, R = ostep.factor_ema(hp.init_scale * np.eye(br), hp.init_scale * np.eye(bc), Gb, hp.beta)
         kap = max(kappa(L + hp.eps * np.eye(br)), kappa(R + hp.eps * np.eye(bc)))
-        tol = UPDATE_TOL * max(1.0, kap / KAPPA_REGIME)
-        rows.append((k, br, bc, kap, rel(d_gpu, d_ref), tol))
-    assert rows
+        rows.append((k, br, bc, kap, rel(d_gpu, d_ref)))
+    assert len(rows) >= min(n_sample, len(table)) - 1
     if require_regime:
         assert all(r[3] <= KAPPA_REGIME for r in rows), rows
-    assert all(r[4] < r[5] for r in rows), rows
+    worst = max(rows, key=lambda r: r[4])
+    print(f"B={B} {solver}: {len(rows)} blocks, worst update error {worst[4]:.2e} (block {worst[0]}, "
+          f"{worst[1]}x{worst[2]}, kappa {worst[3]:.1e}); kappa up to {max(r[3] for r in rows):.1e}")
+    assert all(r[4] < UPDATE_TOL for r in rows), [r for r in rows if r[4] >= UPDATE_TOL]
     return rows
 
 
@@ -89,27 +109,34 @@ def test_gpt2_124m_b512(torch):
 def test_llama_1b_b1024(torch):
     shapes = workloads.llama_1b_shapes()
     grads = workloads.torch_gaussian_gradients(shapes, "cuda", std=0.1, seed=0, row_lognormal_sigma=1.0)
-    run_and_check(torch, shapes, grads, 1024, n_sample=5)
+    run_and_check(torch, shapes, grads, 1024)
 
 
 @pytest.mark.parametrize("B", [128, 256, 512, 1024, 2048])
 def test_mixed_shapes_block_sweep(torch, B):
     shapes = workloads.mixed_shapes()
     grads = workloads.torch_student_t_gradients(shapes, "cuda", nu=3.0, seed=0)
-    run_and_check(torch, shapes, grads, B, n_sample=4)
+    run_and_check(torch, shapes, grads, B)
 
 
-@pytest.mark.parametrize("B", [512, 2048])
-def test_mixed_shapes_chebyshev(torch, B):
+@pytest.mark.parametrize("B,degree", [(512, 16), (2048, 16), (1024, 60), (2048, 60)])
+def test_mixed_shapes_chebyshev(torch, B, degree):
+    # degree 60 is the explainer's figure for the Chebyshev solver
     shapes = workloads.mixed_shapes()
     grads = workloads.torch_student_t_gradients(shapes, "cuda", nu=3.0, seed=1)
-    run_and_check(torch, shapes, grads, B, solver="cheb", degree=16, n_sample=4)
+    run_and_check(torch, shapes, grads, B, solver="cheb", degree=degree)
+
+
+def test_llama_1b_b1024_chebyshev_d60(torch):
+    shapes = workloads.llama_1b_shapes()
+    grads = workloads.torch_gaussian_gradients(shapes, "cuda", std=0.1, seed=0, row_lognormal_sigma=1.0)
+    run_and_check(torch, shapes, grads, 1024, solver="cheb", degree=60)
 
 
 @pytest.mark.parametrize("B", [256, 1024, 2048])
 def test_mixed_shapes_in_regime(torch, B):
-    # root-time damping eps = 1e-2 bounds every factor's condition number by
-    # 1e6 here, so every sampled block is held to the stated 5e-3
+    # root-time damping eps = 3e-2 bounds every factor's condition number by
+    # 1e6 here, the regime the root tolerance is stated for
     shapes = workloads.mixed_shapes()
     grads = workloads.torch_student_t_gradients(shapes, "cuda", nu=3.0, seed=2)
-    run_and_check(torch, shapes, grads, B, n_sample=4, eps=1e-2, require_regime=True)
+    run_and_check(torch, shapes, grads, B, eps=3e-2, require_regime=True)

@@ -224,3 +224,33 @@ def test_coupled_newton_step(torch):
     hp = ostep.HParams(block_size=128, solver="cn", cn_iters=18, eps=1e-4)
     gpu = run_gpu(torch, th, grads, hp)
     compare(gpu, th, grads, hp)
+
+
+@pytest.mark.parametrize("sigma", [1e-8, 1e-4, 1e3])
+def test_gradient_scales(torch, sigma):
+    # gradients far from unit scale: each block is gathered scaled by an exact
+    # power of two (its entries then lie in (-1, 1)), so the split-fp16
+    # products neither underflow (sigma = 1e-8: entries below the fp16 normal
+    # range) nor overflow; eps and the initial factors scale with sigma^2 so
+    # the factors keep the conditioning of the sigma = 0.1 tests
+    shapes = [(256, 384), (200, 130)]
+    grads = [[g * (sigma / 0.1)] for g in workloads.gaussian_gradients(shapes, std=0.1, seed=30)]
+    th = workloads.parameters(shapes, seed=31)
+    reg = 1e-6 * (sigma / 0.1) ** 2
+    hp = ostep.HParams(block_size=128, ndb_iters1=14, ndb_iters2=14, eps=reg, init_scale=reg)
+    gpu = run_gpu(torch, th, grads, hp)
+    compare(gpu, th, grads, hp)
+
+
+def test_gradient_entries_beyond_fp16_range(torch):
+    # gradients N(0, (2e4)^2): about one entry in a thousand lies above the
+    # largest fp16 value (65504); the block's power-of-two scaling keeps every
+    # entry in range, status stays clean, and the step matches the oracle
+    shapes = [(256, 256), (128, 200)]
+    grads = [[g * (2e4 / 0.1)] for g in workloads.gaussian_gradients(shapes, std=0.1, seed=32)]
+    assert max(np.abs(g[0]).max() for g in grads) > 65504.0
+    th = workloads.parameters(shapes, seed=34)
+    reg = 1e-6 * (2e4 / 0.1) ** 2
+    hp = ostep.HParams(block_size=128, ndb_iters1=14, ndb_iters2=14, eps=reg, init_scale=reg)
+    gpu = run_gpu(torch, th, grads, hp)
+    compare(gpu, th, grads, hp)

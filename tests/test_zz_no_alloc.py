@@ -5,8 +5,9 @@ host framework that owns all device memory): its scratch is a fixed array in
 the library's device memory instead of a caller workspace.  This test calls it
 through the C ABI twice in a row, on different inputs, and checks each result
 against the workspace entry point shampoo_inv_root_newton_db on the same
-inputs, within the root tolerance the other GPU tests use.  It also checks
-that a problem larger than the scratch is rejected.  The file is named to be
+inputs, within the root tolerance the other GPU tests use, and reads the
+status word the entry point keeps in its scratch after each call.  It also
+checks that a problem larger than the scratch is rejected.  The file is named to be
 collected last so that a run stopping at the first failure has already run
 every other test.
 """
@@ -49,6 +50,8 @@ def test_static_scratch_matches_workspace_entry_point(torch):
         At = torch.from_numpy(A).cuda()
         rc, X, lam = call_static(torch, lib, At, vt, it, stream)
         assert rc == bd.SHAMPOO_OK, (call, bd.strerror(rc))
+        # the scratch's status word reports a clean call
+        assert bd.read_static_status() == (bd.SHAMPOO_OK, 0)
         torch.cuda.synchronize()
         Xw, lamw, ws = bd.inv_root_newton_db(At, vt, iters1=it, iters2=it, eps=1e-6, pi_iters=10)
         assert bd.read_status(ws)[0] == bd.SHAMPOO_OK

@@ -37,18 +37,18 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
 }
 
 __device__ __forceinline__ void store_split16(__half* base, size_t BB, size_t idx, const float* v, bool& bad) {
-  __half hi[16], lo[16];
+  __half2 hi[8], lo[8];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    split_f16(v[j], hi[j], lo[j]);
-    bad |= (__hisinf(hi[j]) != 0);
+  for (int j = 0; j < 8; ++j) {
+    split_f16x2(v[2 * j], v[2 * j + 1], hi[j], lo[j]);
+    bad |= f16_overflows(v[2 * j]) || f16_overflows(v[2 * j + 1]);
   }
   uint4* dh = reinterpret_cast<uint4*>(base + idx);
   uint4* dl = reinterpret_cast<uint4*>(base + BB + idx);
-  dh[0] = *reinterpret_cast<const uint4*>(&hi[0]);
-  dh[1] = *reinterpret_cast<const uint4*>(&hi[8]);
+  dh[0] = *reinterpret_cast<const uint4*>(&hi[0]);  // hi[0..3]: columns 0..7
+  dh[1] = *reinterpret_cast<const uint4*>(&hi[4]);  // hi[4..7]: columns 8..15
   dl[0] = *reinterpret_cast<const uint4*>(&lo[0]);
-  dl[1] = *reinterpret_cast<const uint4*>(&lo[8]);
+  dl[1] = *reinterpret_cast<const uint4*>(&lo[4]);
 }
 
 // out(col0 + j, row) = v[j]: for a fixed j the 32 lanes (consecutive rows)
@@ -56,12 +56,14 @@ __device__ __forceinline__ void store_split16(__half* base, size_t BB, size_t id
 __device__ __forceinline__ void store_split16_t(__half* base, size_t B, size_t BB, int row, int col0, const float* v,
                                                 bool& bad) {
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    __half h, l;
-    split_f16(v[j], h, l);
-    bad |= (__hisinf(h) != 0);
-    base[(col0 + j) * B + row] = h;
-    base[BB + (col0 + j) * B + row] = l;
+  for (int j = 0; j < 16; j += 2) {
+    __half2 h, l;
+    split_f16x2(v[j], v[j + 1], h, l);
+    bad |= f16_overflows(v[j]) || f16_overflows(v[j + 1]);
+    base[(col0 + j) * B + row] = __low2half(h);
+    base[(col0 + j + 1) * B + row] = __high2half(h);
+    base[BB + (col0 + j) * B + row] = __low2half(l);
+    base[BB + (col0 + j + 1) * B + row] = __high2half(l);
   }
 }
 

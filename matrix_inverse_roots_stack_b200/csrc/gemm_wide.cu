@@ -341,18 +341,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool mirror = args.sym && q > ti;
       GemmEpilogue ep;
       ep.init(g, p, B, BB);
-      GemmEpilogue::CinRaw nxt;  // Cin one chunk ahead (from L2 by now)
-      if (write && ep.has_cin()) nxt = ep.load_cin(B, BB, row, cbase);
+      // Cin streams two 16-column chunks ahead of use (L2 hits by now); a
+      // deeper ring would not fit the accumulator warps' registers
+      constexpr int kAhead = 2;
+      GemmEpilogue::CinRaw pre[kAhead];
+      const bool cin = write && ep.has_cin();
+      if (cin) {
+#pragma unroll
+        for (int c = 0; c < kAhead; ++c) pre[c] = ep.load_cin(B, BB, row, cbase + 16 * c);
+      }
 #pragma unroll 1
-      for (int c = 0; c < (write ? kCols / 16 : 0); ++c) {
+      for (int c = 0; c < (write ? kCols / 16 : 0); ++c) {  // pre[0] holds chunk c; the ring rotates
         const int col0 = cbase + c * 16;
         float v[16], cj[16];
         tmem_ld_32x32b_x16(src + 16 * c, reinterpret_cast<uint32_t*>(v));
         tmem_ld_wait();
-        if (ep.has_cin()) {
-          const GemmEpilogue::CinRaw cur = nxt;
-          if (c + 1 < kCols / 16) nxt = ep.load_cin(B, BB, row, col0 + 16);
-          ep.join_cin(cur, cj);
+        if (cin) {
+          ep.join_cin(pre[0], cj);
+#pragma unroll
+          for (int i = 0; i + 1 < kAhead; ++i) pre[i] = pre[i + 1];
+          if (c + kAhead < kCols / 16) pre[kAhead - 1] = ep.load_cin(B, BB, row, col0 + 16 * kAhead);
         }
         ep.chunk(g, B, BB, row, col0, v, cj, mirror);
       }

@@ -44,9 +44,9 @@ __global__ void frob_norm_kernel(const float* __restrict__ F, int B, float eps, 
 // ------------------------------------------------------------ solver prologues
 
 __device__ __forceinline__ void store_split4(__half* base, size_t BB, size_t idx, const float* x) {
-  __half h[4], l[4];
+  __half2 h[2], l[2];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) split_f16(x[e], h[e], l[e]);
+  for (int e = 0; e < 2; ++e) split_f16x2(x[2 * e], x[2 * e + 1], h[e], l[e]);
   *reinterpret_cast<uint2*>(base + idx) = *reinterpret_cast<const uint2*>(h);
   *reinterpret_cast<uint2*>(base + BB + idx) = *reinterpret_cast<const uint2*>(l);
 }
@@ -54,10 +54,14 @@ __device__ __forceinline__ void store_split4(__half* base, size_t BB, size_t idx
 __device__ __forceinline__ void load_split4(const __half* base, size_t BB, size_t idx, float* x) {
   const uint2 a = *reinterpret_cast<const uint2*>(base + idx);
   const uint2 b = *reinterpret_cast<const uint2*>(base + BB + idx);
-  const __half* h = reinterpret_cast<const __half*>(&a);
-  const __half* l = reinterpret_cast<const __half*>(&b);
+  const __half2* h = reinterpret_cast<const __half2*>(&a);
+  const __half2* l = reinterpret_cast<const __half2*>(&b);
 #pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = join_f16(h[e], l[e]);
+  for (int e = 0; e < 2; ++e) {
+    const float2 fh = __half22float2(h[e]), fl = __half22float2(l[e]);
+    x[2 * e] = fh.x + fl.x * kLoUnscale;
+    x[2 * e + 1] = fh.y + fl.y * kLoUnscale;
+  }
 }
 
 // Newton-DB prologues (element-wise; grid (B*B/1024, nf), 256 threads, 4

@@ -266,4 +266,18 @@ __device__ __forceinline__ float join_f16(__half hi, __half lo) {
   return __half2float(hi) + __half2float(lo) * kLoUnscale;
 }
 
+// The same split of two floats with packed conversions (two-wide
+// float->half and half->float instructions, the same round-to-nearest
+// results): the element-wise conversions are the costly part of writing a
+// split tile.
+__device__ __forceinline__ void split_f16x2(float x0, float x1, __half2& hi, __half2& lo) {
+  hi = __float22half2_rn(make_float2(x0, x1));
+  const float2 b = __half22float2(hi);
+  lo = __float22half2_rn(make_float2((x0 - b.x) * kLoScale, (x1 - b.y) * kLoScale));
+}
+
+// True when x's hi plane would overflow fp16 (|x| rounds to at least
+// 65520) or x is not finite.
+__device__ __forceinline__ bool f16_overflows(float x) { return !(fabsf(x) < 65520.0f); }
+
 }  // namespace dash

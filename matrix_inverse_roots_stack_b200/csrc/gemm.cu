@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x16(src + 32 * c, r);
           tmem_ld_32x32b_x16(src + 32 * c + 16, r + 16);
-          tmem_ld_wait();
+          tmem_ld_wait_regs<32>(r);
           if (c + 1 == kCols / 32) {  // registers hold the whole step now
             tc_fence_before();
             __syncwarp();
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int col0 = cbase + c * 16;
         float v[16], cj[16];
         tmem_ld_32x32b_x16(tbase + lane_off + kColPark + 16 * c, reinterpret_cast<uint32_t*>(v));
-        tmem_ld_wait();
+        tmem_ld_wait_regs<16>(reinterpret_cast<uint32_t*>(v));
         if (c + 1 == kTile / 16) {  // the park buffer is free for the next tile
           tc_fence_before();
           __syncwarp();

@@ -173,9 +173,9 @@ struct GemmEpilogue {
     }
   }
 
-  // One 16-column chunk; cj holds Cin's chunk in fp32 when has_cin().
-  __device__ __forceinline__ void chunk(const GemmOp& g, size_t B, size_t BB, int row, int col0, float* v,
-                                        const float* cj, bool mirror) {
+  // v = s_p * (alpha * a_p * acc + beta * Cin + gamma * I) for one
+  // 16-column chunk; cj holds Cin's chunk in fp32 when has_cin().
+  __device__ __forceinline__ void apply(int row, int col0, float* v, const float* cj) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] *= alpha;
     if (has_cin()) {
@@ -193,16 +193,43 @@ struct GemmEpilogue {
       v[j] *= s;
       bad |= !isfinite(v[j]);
     }
-    if (scatter) {
-      if (row < bd.br) {
-        float* dst = g.u_out + bd.off + static_cast<long long>(bd.r0 + row) * bd.pitch + bd.c0 + col0;
+  }
+
+  // Scatter of an applied chunk into parameter layout (rows and columns
+  // past the block's extent are dropped), with its sum of squares.
+  __device__ __forceinline__ void scatter_chunk(const GemmOp& g, int row, int col0, const float* v) {
+    if (row >= bd.br) return;
+    float* dst = g.u_out + bd.off + static_cast<long long>(bd.r0 + row) * bd.pitch + bd.c0 + col0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (col0 + j < bd.bc) {
-            dst[j] = v[j];
-            sumsq += v[j] * v[j];
-          }
+    for (int j = 0; j < 16; ++j)
+      if (col0 + j < bd.bc) {
+        dst[j] = v[j];
+        sumsq += v[j] * v[j];
       }
+  }
+
+  // Transposed copy of an applied chunk (symmetric launches): for a fixed
+  // column the 32 lanes (consecutive rows) write consecutive addresses.
+  __device__ __forceinline__ void store_mirror(size_t B, size_t BB, int row, int col0, const float* v) {
+    if (os) {
+      float w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) w[j] = v[j] * ss;
+      store_split16_t(os, B, BB, row, col0, w, bad);
+    }
+    if (of) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) of[(col0 + j) * B + row] = v[j];
+    }
+  }
+
+  // One 16-column chunk written straight from registers (row-major split
+  // and/or fp32, plus the mirror), or scattered.
+  __device__ __forceinline__ void chunk(const GemmOp& g, size_t B, size_t BB, int row, int col0, float* v,
+                                        const float* cj, bool mirror) {
+    apply(row, col0, v, cj);
+    if (scatter) {
+      scatter_chunk(g, row, col0, v);
       return;
     }
     if (os) {
@@ -210,17 +237,13 @@ struct GemmEpilogue {
 #pragma unroll
       for (int j = 0; j < 16; ++j) w[j] = v[j] * ss;
       store_split16(os, BB, row * B + col0, w, bad);
-      if (mirror) store_split16_t(os, B, BB, row, col0, w, bad);
     }
     if (of) {
       float4* d4 = reinterpret_cast<float4*>(of + row * B + col0);
 #pragma unroll
       for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      if (mirror) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) of[(col0 + j) * B + row] = v[j];
-      }
     }
+    if (mirror) store_mirror(B, BB, row, col0, v);
   }
 
   // Warp-collective: the non-finite flag and the scattered sum of squares.

@@ -2,15 +2,25 @@
 // launches whose block size is a multiple of 256 (split-fp16 products;
 // symmetric launches take the tiles that reach the upper triangle).
 //
-// Same arithmetic as gemm.cu (per K=16 step: hi*lo + lo*hi into a fresh
-// tensor-memory buffer, then hi*hi with that buffer scaled by 2^-11, the
-// step's product added into fp32 registers with round-to-nearest), with a
-// tile twice as wide.  Every MMA issues as much tensor work as it can
-// (M=128, N=256), so a step carries twice the work of a 128 x 128 tile for
-// the same issue, barrier and hand-off overhead; the price is tensor memory:
-// a step's fp32 product takes 256 of the 512 columns, so the ring holds two
-// steps and there is no room to park a finished tile.  The accumulator
+// Split-fp16 products as in gemm.cu (hi*lo + lo*hi into a fresh
+// tensor-memory buffer, then hi*hi with that buffer scaled by 2^-11), with a
+// tile twice as wide and one buffer per two K=16 steps instead of per step:
+// the buffer takes the cross terms of both steps, then hi*hi of the first
+// step plus 2^-11 times them, then hi*hi of the second, and the buffer's fp32
+// product is added into fp32 registers with round-to-nearest.  Every
+// tensor-core accumulation rounds toward zero once per MMA, relative to the
+// running partial sum in the buffer; with two steps per buffer that partial
+// is at most twice a step's, which measured within 10% of per-step adds on
+// the update error of blocks with condition numbers near 1e8, while four
+// steps per buffer raised it by about 1.7x.  Two steps halve the register
+// flush work (loads from tensor memory and fp32 adds) per product.
+// Every MMA issues as much tensor work as it can (M=128, N=256); a buffer's
+// fp32 product takes 256 of the 512 tensor-memory columns, so the ring holds
+// two buffers and there is no room to park a finished tile.  The accumulator
 // warps therefore write their own tile out.
+//
+// Shared memory: two 96 KB operand stages, 32 KB of epilogue staging, the
+// barriers (about 225 KB of the 227 KB a block may hold).
 //
 // Roles (384 threads = three warpgroups, one CTA per SM, persistent over a
 // static round-robin list of the launch's tiles):
@@ -18,13 +28,17 @@
 //                      lanes 32*(w%4).. and 128 of the 256 columns, so each
 //                      thread sums 128 columns of one output row in
 //                      registers; at the end of a tile the same thread applies
-//                      the epilogue to its row segment and stores it.
+//                      the epilogue to its row segment.  Row-major outputs
+//                      leave through the warp's two 2 KB shared-memory
+//                      staging buffers, one TMA tensor store per 32 x 16
+//                      chunk (a store instruction whose 32 lanes each write
+//                      a different row would touch 32 lines).
 //   warp 8, one lane   TMA producer: A hi/lo (128 x 64) and B hi/lo
 //                      (256 x 64, or four 64 x 64 boxes when B is read
 //                      MN-major) of each 64-wide K slab into a 2-stage ring
 //                      of 96 KB stages.  No multicast.
-//   warp 9, one lane   MMA issuer: three tcgen05.mma kind::f16 per K=16 step
-//                      into one of two 256-column tensor-memory buffers.
+//   warp 9, one lane   MMA issuer: six tcgen05.mma kind::f16 per two K=16
+//                      steps into one of two 256-column tensor-memory buffers.
 //   warps 10-11        idle (they complete warpgroup 2).
 // Register split: the kernel is launched at 168 registers a thread (384 x
 // 168 = 64,512 of the SM's 65,536); warpgroup 2 gives registers back with
@@ -41,6 +55,7 @@
 #include "tmap.cuh"
 
 #include <atomic>
+#include <cstring>
 
 namespace dash {
 namespace {
@@ -51,7 +66,11 @@ constexpr int kABytes = kM * kKBlk * 2;                // 16 KB per plane and sl
 constexpr int kBBytes = kN * kKBlk * 2;                // 32 KB per plane and slab
 constexpr int kStageBytes = 2 * kABytes + 2 * kBBytes;  // A hi, A lo, B hi, B lo
 constexpr int kStages = 2;
-constexpr int kRing = 2;                               // per-K-step product buffers of kN columns
+constexpr int kRing = 2;                               // product buffers of kN columns
+constexpr int kFillSteps = 2;                          // K=16 steps a buffer takes before its flush
+constexpr int kFills = kKBlk / 16 / kFillSteps;        // buffer fills per K slab
+static_assert(kFills * kFillSteps * 16 == kKBlk, "fills must tile the K slab");
+constexpr int kChunk = 32;                             // columns per tensor-memory load batch of a flush
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAccWarps = 8;                           // warps 0-7
 constexpr int kProdWarp = 8, kMmaWarp = 9;
@@ -61,8 +80,7 @@ constexpr int kLowRegs = 72, kHighRegs = 216;          // after setmaxnreg: warp
 static_assert(2 * 128 * kHighRegs + 128 * kLowRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
 static_assert(2 * 32 * kHighRegs + 32 * kLowRegs <= 16384, "register split exceeds a scheduler's file");
 constexpr int kCols = 128;                             // columns summed per accumulator thread
-constexpr int kPrefetchSteps = 6;                      // K=16 steps before a tile's end when its Cin is prefetched
-constexpr int kChunk = 32;                             // columns per tensor-memory load batch
+constexpr int kPrefetchSlabs = 2;                      // 64-wide K slabs before a tile's end when its Cin is prefetched
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
@@ -71,7 +89,20 @@ struct Bars {
   uint32_t tmem_slot;
   int abort;
 };
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + static_cast<int>(sizeof(Bars)) + 64;
+// Epilogue staging: per accumulator warp two 2 KB buffers, each one 32 x 16
+// chunk of split output (both planes) or of fp32 output, written by the
+// warp in the TMA swizzle and stored with one tensor store.
+constexpr int kStageBufBytes = 2048;
+constexpr int kStagingOff = kStages * kStageBytes;
+constexpr int kBarsOff = kStagingOff + kAccWarps * 2 * kStageBufBytes;
+constexpr int kSmemBytes = kBarsOff + 1024 + static_cast<int>(sizeof(Bars)) + 64;
+static_assert(kSmemBytes <= 232448, "shared memory exceeds the per-block limit");
+
+// Output tensor maps of a launch: split and fp32 outputs of op 0 and op 1
+// (encoded for the outputs an op has, unless it scatters).
+struct OutMaps {
+  CUtensorMap split[2], f32[2];
+};
 
 // Tiles of one problem.  Symmetric launches take the 128 x 256 tiles that
 // reach the upper triangle, 2 tj + 1 >= ti in 128-column units: row ti has
@@ -133,21 +164,72 @@ __device__ __forceinline__ void prefetch_cin_l2(const GemmOp& g, int p, size_t B
   }
 }
 
+// Staging writes: lane l holds row l of a 32 x 16 chunk.  Split chunk:
+// plane k (hi, lo) at k * 1 KB, row l at 32 l, its two 16-byte halves
+// swapped when bit 2 of l is set (32-byte swizzle: address bit 4 ^= bit 7).
+// fp32 chunk: row l at 64 l, 16-byte quarter h at h ^ ((l >> 1) & 3)
+// (64-byte swizzle: bits 5:4 ^= bits 8:7).  Eight consecutive lanes cover
+// all 32 banks, so each 16-byte store takes the minimum four wavefronts.
+__device__ __forceinline__ void stage_split16(uint8_t* buf, int lane, const float* w, bool& bad) {
+  __half2 hi[8], lo[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    split_f16x2(w[2 * j], w[2 * j + 1], hi[j], lo[j]);
+    bad |= f16_overflows(w[2 * j]) || f16_overflows(w[2 * j + 1]);
+  }
+  const int x = (lane >> 2) & 1;
+  uint8_t* r = buf + lane * 32;
+  *reinterpret_cast<uint4*>(r + 16 * x) = *reinterpret_cast<const uint4*>(&hi[0]);
+  *reinterpret_cast<uint4*>(r + 16 * (x ^ 1)) = *reinterpret_cast<const uint4*>(&hi[4]);
+  *reinterpret_cast<uint4*>(r + 1024 + 16 * x) = *reinterpret_cast<const uint4*>(&lo[0]);
+  *reinterpret_cast<uint4*>(r + 1024 + 16 * (x ^ 1)) = *reinterpret_cast<const uint4*>(&lo[4]);
+}
+
+__device__ __forceinline__ void stage_f32x16(uint8_t* buf, int lane, const float* v) {
+  const int x = (lane >> 1) & 3;
+  uint8_t* r = buf + lane * 64;
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+    *reinterpret_cast<float4*>(r + 16 * (h ^ x)) = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
+}
+
+// A warp's staging ring: before a buffer is rewritten, the tensor store
+// issued from it two stores ago must have finished reading it.
+struct StageRing {
+  uint8_t* base;  // this warp's two buffers
+  int next;
+  __device__ __forceinline__ uint8_t* acquire(int lane) {
+    if (lane == 0) bulk_wait_read<1>();
+    __syncwarp();
+    return base + next * kStageBufBytes;
+  }
+  // the warp's writes to buf go out as one tensor store at (c0, c1, c2)
+  __device__ __forceinline__ void release(int lane, const CUtensorMap* map, const uint8_t* buf, int c0, int c1,
+                                          int c2) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(map, buf, c0, c1, c2);
+      bulk_commit();
+    }
+    next ^= 1;
+  }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                     const GemmArgs args, const long long total) {
+                     const __grid_constant__ OutMaps om, const GemmArgs args, const long long total) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  Bars* bars = reinterpret_cast<Bars*>(smem + kBarsOff);
   volatile int* abort_flag = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = args.B / kN;
   const int tpp = wide_tiles_per_problem(args.B, args.sym);
   const int nk = args.B / kKBlk;
-  const int nsteps = nk * (kKBlk / 16);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -244,16 +326,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t so = s * (kStageBytes >> 4);
           const uint64_t ah = kd0 + so, al = ah + kAD, bh = bd0 + so, bl = bh + kBD;
 #pragma unroll
-          for (int kk = 0; kk < kKBlk / 16; ++kk) {
+          for (int f = 0; f < kFills; ++f) {
             ok = mbar_wait(&bars->acc_empty[hb], (hpar >> hb) & 1u, abort_flag);
             hpar ^= 1u << hb;
             if (!ok) break;
             tc_fence_after();
-            const uint32_t ka = 2u * kk, kbo = bstep * kk;
             const uint32_t d = tbase + hb * kN;
-            mma_f16_ss(d, ah + ka, bl + kbo, idesc, 0u);         // hi * lo
-            mma_f16_ss(d, al + ka, bh + kbo, idesc, 1u);         // + lo * hi
-            mma_f16_ss_acc_down11(d, ah + ka, bh + kbo, idesc);  // hi * hi + 2^-11 * (...)
+            const int k0 = f * kFillSteps;
+            // cross terms hi*lo + lo*hi of the fill's K=16 steps into a fresh
+            // buffer, then hi*hi of its first step plus 2^-11 times that sum,
+            // then hi*hi of its other steps
+#pragma unroll
+            for (int kk = k0; kk < k0 + kFillSteps; ++kk) {
+              mma_f16_ss(d, ah + 2u * kk, bl + bstep * kk, idesc, kk > k0 ? 1u : 0u);
+              mma_f16_ss(d, al + 2u * kk, bh + bstep * kk, idesc, 1u);
+            }
+            mma_f16_ss_acc_down11(d, ah + 2u * k0, bh + bstep * k0, idesc);
+#pragma unroll
+            for (int kk = k0 + 1; kk < k0 + kFillSteps; ++kk) mma_f16_ss(d, ah + 2u * kk, bh + bstep * kk, idesc, 1u);
             mma_commit(&bars->acc_full[hb]);
             hb ^= 1u;
           }
@@ -280,21 +370,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t B = static_cast<size_t>(args.B);
     const size_t BB = B * B;
     uint32_t hb = 0, hpar = 0;  // ring buffer, its fill parities
+    StageRing ring{smem + kStagingOff + warp * 2 * kStageBufBytes, 0};
     bool ok = true;
     for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
       float S[kCols];
 #pragma unroll
       for (int j = 0; j < kCols; ++j) S[j] = 0.0f;
-      // Cin of this thread's row segment is fetched into L2 a few steps
+      // Cin of this thread's row segment is fetched into L2 a few slabs
       // before the epilogue needs it (no registers held)
       int op, p, ti, tj;
       decode_wide(args, tpp, ntn, t, op, p, ti, tj);
       const GemmOp& g = args.op[op];
       const int row = ti * kM + quad * 32 + lane;
       const int cbase = tj * kN + cgrp * kCols;
-      const int pf_step = nsteps > kPrefetchSteps ? nsteps - kPrefetchSteps : 0;
-      for (int sg = 0; sg < nsteps; ++sg) {
-        if (sg == pf_step) prefetch_cin_l2(g, p, B, BB, row, cbase);
+      const int nfill = nk * kFills;
+      const int pf_fill = nk > kPrefetchSlabs ? (nk - kPrefetchSlabs) * kFills : 0;
+      // fill sg of the tile: S += its product (the last fill's sums go back
+      // into its buffer for the epilogue instead of releasing it)
+      for (int sg = 0; sg < nfill; ++sg) {
+        if (sg == pf_fill) prefetch_cin_l2(g, p, B, BB, row, cbase);
         // waiting warps sleep in the barrier, leaving the issue slots of
         // their scheduler to the MMA and TMA threads
         if (!mbar_wait_sleep(&bars->acc_full[hb], (hpar >> hb) & 1u, abort_flag)) {
@@ -304,26 +398,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         hpar ^= 1u << hb;
         tc_fence_after();
         const uint32_t src = tbase + lane_off + hb * kN;
-        const bool last = sg + 1 == nsteps;
+        if (sg + 1 < nfill) {
 #pragma unroll
-        for (int c = 0; c < kCols / kChunk; ++c) {
-          uint32_t r[kChunk];
+          for (int c = 0; c < kCols / kChunk; ++c) {
+            uint32_t r[kChunk];
 #pragma unroll
-          for (int q = 0; q < kChunk / 16; ++q) tmem_ld_32x32b_x16(src + kChunk * c + 16 * q, r + 16 * q);
-          tmem_ld_wait();
-          if (!last && c + 1 == kCols / kChunk) {  // registers hold the whole step now
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
+            for (int q = 0; q < kChunk / 16; ++q) tmem_ld_32x32b_x16(src + kChunk * c + 16 * q, r + 16 * q);
+            tmem_ld_wait_regs<kChunk>(r);
+            if (c + 1 == kCols / kChunk) {  // registers hold the whole fill now
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
+            }
+#pragma unroll
+            for (int j = 0; j < kChunk; j += 2) add_f32x2(S[kChunk * c + j], S[kChunk * c + j + 1], r[j], r[j + 1]);
           }
+          hb ^= 1u;
+        } else {
 #pragma unroll
-          for (int j = 0; j < kChunk; j += 2) add_f32x2(S[kChunk * c + j], S[kChunk * c + j + 1], r[j], r[j + 1]);
-          if (last) {  // the tile's sums go back into this buffer for the epilogue
+          for (int c = 0; c < kCols / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(src + 16 * c, r);
+            tmem_ld_wait_regs<16>(r);
 #pragma unroll
-            for (int q = 0; q < kChunk / 16; ++q) tmem_st_32x32b_x16(src + kChunk * c + 16 * q, &S[kChunk * c + 16 * q]);
+            for (int j = 0; j < 16; j += 2) add_f32x2(S[16 * c + j], S[16 * c + j + 1], r[j], r[j + 1]);
+            tmem_st_32x32b_x16(src + 16 * c, &S[16 * c]);
           }
         }
-        if (!last) hb ^= 1u;
       }
       if (!ok) {
         if (lane == 0) gemm_fail_timeout(abort_flag, args.status);
@@ -341,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool mirror = args.sym && q > ti;
       GemmEpilogue ep;
       ep.init(g, p, B, BB);
+      const int row0 = ti * kM + quad * 32;  // first row of this warp's chunks
       // Cin streams two 16-column chunks ahead of use (L2 hits by now); a
       // deeper ring would not fit the accumulator warps' registers
       constexpr int kAhead = 2;
@@ -355,14 +457,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int col0 = cbase + c * 16;
         float v[16], cj[16];
         tmem_ld_32x32b_x16(src + 16 * c, reinterpret_cast<uint32_t*>(v));
-        tmem_ld_wait();
+        tmem_ld_wait_regs<16>(reinterpret_cast<uint32_t*>(v));
         if (cin) {
           ep.join_cin(pre[0], cj);
 #pragma unroll
           for (int i = 0; i + 1 < kAhead; ++i) pre[i] = pre[i + 1];
           if (c + kAhead < kCols / 16) pre[kAhead - 1] = ep.load_cin(B, BB, row, col0 + 16 * kAhead);
         }
-        ep.chunk(g, B, BB, row, col0, v, cj, mirror);
+        ep.apply(row, col0, v, cj);
+        if (ep.scatter) {
+          ep.scatter_chunk(g, row, col0, v);
+          continue;
+        }
+        // row-major outputs leave through the staging ring (one tensor
+        // store per 32 x 16 chunk instead of 32 row segments per store
+        // instruction); the mirror's stores are already coalesced
+        if (ep.os) {
+          float w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = v[j] * ep.ss;
+          uint8_t* buf = ring.acquire(lane);
+          stage_split16(buf, lane, w, ep.bad);
+          ring.release(lane, &om.split[op], buf, col0, row0, 2 * gemm_at(g.out_i, p));
+        }
+        if (ep.of) {
+          uint8_t* buf = ring.acquire(lane);
+          stage_f32x16(buf, lane, v);
+          ring.release(lane, &om.f32[op], buf, col0, row0, gemm_at(g.outf_i, p));
+        }
+        if (mirror) ep.store_mirror(B, BB, row, col0, v);
       }
       ep.finish(g, p, args.status);
       tc_fence_before();
@@ -370,6 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
       hb ^= 1u;
     }
+    // this warp's tensor stores complete before the CTA's shared memory goes
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -392,6 +517,14 @@ int wide_kernel_regs() {
   return r;
 }
 
+// One past the largest matrix index that problems [0, nprob) of an op
+// reach through i (the host mirror of gemm_at).
+long long idx_extent(const Idx& i, int nprob) {
+  const long long st = i.stride > 0 ? i.stride : 1;
+  const long long n = i.mod > 0 && i.mod < nprob ? i.mod : nprob;
+  return i.base + st * (n - 1) + 1;
+}
+
 }  // namespace
 
 bool gemm_wide_supported(const GemmArgs& a) {
@@ -411,8 +544,23 @@ cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long lo
   // executed tensor-core flops: each 128 x 256 tile is one 2*128*256*B
   // product, done as three fp16 products
   const double flops = 3.0 * 2.0 * kM * kN * static_cast<double>(a.B) * static_cast<double>(total);
+  // output maps over the matrices the launch's problems write
+  OutMaps om;
+  std::memset(&om, 0, sizeof(om));
+  for (int o = 0; o < a.nops; ++o) {
+    const GemmOp& g = a.op[o];
+    if (g.nprob <= 0 || g.blocks) continue;
+    if (g.out_split) {
+      e = encode_epilogue_map(&om.split[o], g.out_split, false, a.B, 2 * idx_extent(g.out_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    }
+    if (g.out_f32) {
+      e = encode_epilogue_map(&om.f32[o], g.out_f32, true, a.B, idx_extent(g.outf_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    }
+  }
   const int slot = prof_begin(kProfGemmWide, stream, flops);
-  gemm_wide_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
+  gemm_wide_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], om, a, total);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

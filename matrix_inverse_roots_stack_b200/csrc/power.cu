@@ -300,7 +300,8 @@ __global__ void __launch_bounds__(kPThreads, 2)
       const uint32_t ta = tbase + (static_cast<uint32_t>(32 * warp) << 16);
       tmem_ld_32x32b_x32(ta, h);
       tmem_ld_32x32b_x32(ta + 32u, x);
-      tmem_ld_wait();
+      tmem_ld_wait_regs<32>(h);
+      tmem_ld_wait_regs<32>(x);
 #pragma unroll
       for (int j = 0; j < kPiStarts; ++j) w[j] = __uint_as_float(h[j]) + __uint_as_float(x[j]) * kLoUnscale;
     }

@@ -44,6 +44,23 @@ cudaError_t encode_f16_3d_map(CUtensorMap* map, const void* base, int cols, int 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_epilogue_map(CUtensorMap* map, void* base, bool f32, int B, long long depth) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return cudaErrorInvalidValue;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0 || B % 32 != 0 || B < 32 || depth < (f32 ? 1 : 2))
+    return cudaErrorInvalidValue;
+  const cuuint64_t esz = f32 ? 4u : 2u;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(B), static_cast<cuuint64_t>(B), static_cast<cuuint64_t>(depth)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(B) * esz, static_cast<cuuint64_t>(B) * B * esz};
+  cuuint32_t box[3] = {16u, 32u, f32 ? 1u : 2u};
+  cuuint32_t estride[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims,
+                   strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   f32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat, int box_rows) {
   if (B % 128 != 0 || nmat < 1) return cudaErrorInvalidValue;
   return encode_f16_3d_map(map, base, B, B, 2ll * nmat, box_rows);

@@ -104,7 +104,7 @@ __device__ __forceinline__ void join_chunk(const SplitChunk& c, float* out) {
 // (mirrored for symmetric launches), or scattered into parameter layout with
 // its sum of squares.
 struct GemmEpilogue {
-  float s, alpha, beta, gamma, ss;
+  float s, alpha, beta, gamma, ss;  // s_p, alpha * a_p, beta, gamma; split-output factor
   const __half* cin;
   const float* cinf;
   __half* os;
@@ -174,25 +174,53 @@ struct GemmEpilogue {
   }
 
   // v = s_p * (alpha * a_p * acc + beta * Cin + gamma * I) for one
-  // 16-column chunk; cj holds Cin's chunk in fp32 when has_cin().
-  __device__ __forceinline__ void apply(int row, int col0, float* v, const float* cj) {
+  // 16-column chunk, in packed fp32 pairs and in this order: alpha a_p acc
+  // (rounded), plus beta Cin (one fused multiply-add), plus gamma on the
+  // diagonal, times s_p.  The order is part of the result: for factors whose
+  // smallest eigenvalues sit near the rounding level of their diagonal (the
+  // exponential moving average of G G^T at condition numbers of 1e7 and
+  // more), folding the scalars into one multiply-add doubled the distance of
+  // the update from the float64 reference.  cj holds Cin's chunk in fp32
+  // when has_cin().  Callers check the result's range (check_finite, or the
+  // fp16 overflow test of the split store, which also catches non-finite
+  // values).
+  __device__ __forceinline__ void apply(int row, int col0, float* v, const float* cj) const {
+    const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] *= alpha;
-    if (has_cin()) {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] += beta * cj[j];
+    for (int j = 0; j < 16; j += 2) {
+      const float2 r = __fmul2_rn(make_float2(v[j], v[j + 1]), a2);
+      v[j] = r.x;
+      v[j + 1] = r.y;
     }
-    if (gamma != 0.0f) {
-      const int d = row - col0;
+    if (has_cin()) {
+      const float2 b2 = make_float2(beta, beta);
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        const float2 r = __ffma2_rn(b2, make_float2(cj[j], cj[j + 1]), make_float2(v[j], v[j + 1]));
+        v[j] = r.x;
+        v[j + 1] = r.y;
+      }
+    }
+    const int d = row - col0;
+    if (gamma != 0.0f && d >= 0 && d < 16) {
 #pragma unroll
       for (int j = 0; j < 16; ++j)
         if (j == d) v[j] += gamma;
     }
+    if (s != 1.0f) {
+      const float2 s2 = make_float2(s, s);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      v[j] *= s;
-      bad |= !isfinite(v[j]);
+      for (int j = 0; j < 16; j += 2) {
+        const float2 r = __fmul2_rn(make_float2(v[j], v[j + 1]), s2);
+        v[j] = r.x;
+        v[j + 1] = r.y;
+      }
     }
+  }
+
+  __device__ __forceinline__ void check_finite(const float* v) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bad |= !isfinite(v[j]);
   }
 
   // Scatter of an applied chunk into parameter layout (rows and columns
@@ -228,6 +256,7 @@ struct GemmEpilogue {
   __device__ __forceinline__ void chunk(const GemmOp& g, size_t B, size_t BB, int row, int col0, float* v,
                                         const float* cj, bool mirror) {
     apply(row, col0, v, cj);
+    if (scatter || of) check_finite(v);
     if (scatter) {
       scatter_chunk(g, row, col0, v);
       return;

@@ -193,26 +193,26 @@ __device__ __forceinline__ void stage_f32x16(uint8_t* buf, int lane, const float
     *reinterpret_cast<float4*>(r + 16 * (h ^ x)) = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
 }
 
-// A warp's staging ring: before a buffer is rewritten, the tensor store
-// issued from it two stores ago must have finished reading it.
-struct StageRing {
-  uint8_t* base;  // this warp's two buffers
-  int next;
-  __device__ __forceinline__ uint8_t* acquire(int lane) {
-    if (lane == 0) bulk_wait_read<1>();
+// A warp's two staging buffers take the two 16-column chunks of one epilogue
+// step; before they are rewritten, the tensor stores issued from them one
+// step earlier must have finished reading them.
+struct Staging {
+  uint8_t* base;
+  __device__ __forceinline__ uint8_t* acquire(int lane) const {
+    if (lane == 0) bulk_wait_read<0>();
     __syncwarp();
-    return base + next * kStageBufBytes;
+    return base;
   }
-  // the warp's writes to buf go out as one tensor store at (c0, c1, c2)
-  __device__ __forceinline__ void release(int lane, const CUtensorMap* map, const uint8_t* buf, int c0, int c1,
-                                          int c2) {
+  // the warp's writes go out as two tensor stores, chunks at (c0, c1, c2)
+  // and (c0 + 16, c1, c2)
+  __device__ __forceinline__ void release(int lane, const CUtensorMap* map, int c0, int c1, int c2) const {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_3d(map, buf, c0, c1, c2);
+      tma_store_3d(map, base, c0, c1, c2);
+      tma_store_3d(map, base + kStageBufBytes, c0 + 16, c1, c2);
       bulk_commit();
     }
-    next ^= 1;
   }
 };
 
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t B = static_cast<size_t>(args.B);
     const size_t BB = B * B;
     uint32_t hb = 0, hpar = 0;  // ring buffer, its fill parities
-    StageRing ring{smem + kStagingOff + warp * 2 * kStageBufBytes, 0};
+    const Staging stg{smem + kStagingOff + warp * 2 * kStageBufBytes};
     bool ok = true;
     for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
       float S[kCols];
@@ -443,49 +443,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       GemmEpilogue ep;
       ep.init(g, p, B, BB);
       const int row0 = ti * kM + quad * 32;  // first row of this warp's chunks
-      // Cin streams two 16-column chunks ahead of use (L2 hits by now); a
-      // deeper ring would not fit the accumulator warps' registers
-      constexpr int kAhead = 2;
-      GemmEpilogue::CinRaw pre[kAhead];
+      // each step takes two 16-column chunks (one tensor-memory wait, one
+      // staging round); Cin streams one step ahead of use (L2 hits by now;
+      // a deeper ring does not fit the accumulator warps' registers)
+      GemmEpilogue::CinRaw pre[2];
       const bool cin = write && ep.has_cin();
       if (cin) {
-#pragma unroll
-        for (int c = 0; c < kAhead; ++c) pre[c] = ep.load_cin(B, BB, row, cbase + 16 * c);
+        pre[0] = ep.load_cin(B, BB, row, cbase);
+        pre[1] = ep.load_cin(B, BB, row, cbase + 16);
       }
 #pragma unroll 1
-      for (int c = 0; c < (write ? kCols / 16 : 0); ++c) {  // pre[0] holds chunk c; the ring rotates
+      for (int c = 0; c < (write ? kCols / 16 : 0); c += 2) {  // pre[0..1] hold chunks c, c+1
         const int col0 = cbase + c * 16;
-        float v[16], cj[16];
-        tmem_ld_32x32b_x16(src + 16 * c, reinterpret_cast<uint32_t*>(v));
-        tmem_ld_wait_regs<16>(reinterpret_cast<uint32_t*>(v));
-        if (cin) {
-          ep.join_cin(pre[0], cj);
+        float v[2][16];
+        tmem_ld_32x32b_x16(src + 16 * c, reinterpret_cast<uint32_t*>(v[0]));
+        tmem_ld_32x32b_x16(src + 16 * c + 16, reinterpret_cast<uint32_t*>(v[1]));
+        tmem_ld_wait_regs<32>(reinterpret_cast<uint32_t*>(v));
 #pragma unroll
-          for (int i = 0; i + 1 < kAhead; ++i) pre[i] = pre[i + 1];
-          if (c + kAhead < kCols / 16) pre[kAhead - 1] = ep.load_cin(B, BB, row, col0 + 16 * kAhead);
+        for (int h = 0; h < 2; ++h) {
+          float cj[16];
+          if (cin) {
+            ep.join_cin(pre[h], cj);
+            if (c + 2 < kCols / 16) pre[h] = ep.load_cin(B, BB, row, col0 + 32 + 16 * h);
+          }
+          ep.apply(row, col0 + 16 * h, v[h], cj);
         }
-        ep.apply(row, col0, v, cj);
         if (ep.scatter) {
-          ep.scatter_chunk(g, row, col0, v);
+          ep.check_finite(v[0]);
+          ep.check_finite(v[1]);
+          ep.scatter_chunk(g, row, col0, v[0]);
+          ep.scatter_chunk(g, row, col0 + 16, v[1]);
           continue;
         }
-        // row-major outputs leave through the staging ring (one tensor
+        // row-major outputs leave through the staging buffers (one tensor
         // store per 32 x 16 chunk instead of 32 row segments per store
         // instruction); the mirror's stores are already coalesced
         if (ep.os) {
-          float w[16];
+          uint8_t* buf = stg.acquire(lane);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) w[j] = v[j] * ep.ss;
-          uint8_t* buf = ring.acquire(lane);
-          stage_split16(buf, lane, w, ep.bad);
-          ring.release(lane, &om.split[op], buf, col0, row0, 2 * gemm_at(g.out_i, p));
+          for (int h = 0; h < 2; ++h) {
+            float w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = v[h][j] * ep.ss;
+            stage_split16(buf + h * kStageBufBytes, lane, w, ep.bad);
+          }
+          stg.release(lane, &om.split[op], col0, row0, 2 * gemm_at(g.out_i, p));
         }
         if (ep.of) {
-          uint8_t* buf = ring.acquire(lane);
-          stage_f32x16(buf, lane, v);
-          ring.release(lane, &om.f32[op], buf, col0, row0, gemm_at(g.outf_i, p));
+          ep.check_finite(v[0]);
+          ep.check_finite(v[1]);
+          uint8_t* buf = stg.acquire(lane);
+          stage_f32x16(buf, lane, v[0]);
+          stage_f32x16(buf + kStageBufBytes, lane, v[1]);
+          stg.release(lane, &om.f32[op], col0, row0, gemm_at(g.outf_i, p));
         }
-        if (mirror) ep.store_mirror(B, BB, row, col0, v);
+        if (mirror) {
+          ep.store_mirror(B, BB, row, col0, v[0]);
+          ep.store_mirror(B, BB, row, col0 + 16, v[1]);
+        }
       }
       ep.finish(g, p, args.status);
       tc_fence_before();

@@ -41,13 +41,14 @@ sys.path.insert(0, ROOT)
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 
-# DRAM bytes (read + write) per executed tensor-core flop of gemm_split_kernel,
-# by (block size, solver): from an ncu capture of every GEMM launch of one step
-# of the mixed-shape B=1024 workload (24 factors of 1024, Newton-DB 14 + 14).
-# Each launch reads and writes its problems' split matrices about once, so a
-# launch's traffic grows in proportion to the problems, and executed flops, it
-# covers; the roofline's per-launch traffic scales this ratio by those flops.
-GEMM_DRAM_BYTES_PER_FLOP = {(1024, "ndb"): 1.606e-3}
+# DRAM bytes (read + write) per executed tensor-core flop of the GEMM, by
+# (kernel, block size, solver): from an ncu capture of every launch of three
+# steps of the mixed-shape B=1024 workload (24 factors of 1024, Newton-DB
+# 14 + 14): 59.85 GB over 3.69e13 executed flops.  Each launch reads and writes
+# its problems' split matrices about once, so a launch's traffic grows in
+# proportion to the problems, and executed flops, it covers; the roofline's
+# per-launch traffic scales this ratio by those flops.
+GEMM_DRAM_BYTES_PER_FLOP = {("gemm_wide_kernel", 1024, "ndb"): 1.621e-3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -557,8 +558,7 @@ def main():
     name = max(kernels, key=lambda k: kernels[k][0])
     g_ms, g_n, g_flops = kernels[name]
     avg_ms, achieved = kernel_line(g_ms, g_n, g_flops)
-    # DRAM bytes per executed flop were captured on the 128 x 128 kernel
-    bpf = GEMM_DRAM_BYTES_PER_FLOP.get((B, args.solver)) if name == "gemm_split_kernel" else None
+    bpf = GEMM_DRAM_BYTES_PER_FLOP.get((name, B, args.solver))
     traffic = round(bpf * g_flops / g_n) if (bpf and g_n) else None
     roofline = {"kernel": name, "bound": "tensor",
                 "achieved": round(achieved, 1) if achieved else None, "peak": tensor_peak,

@@ -60,7 +60,8 @@ struct GemmOp {
   int split_norm;            // 1: the split output is out_p * 2^-e with 2^(e-1) <= s_p < 2^e
   float* out_f32;            // fp32 output (+ mirror if sym)
   Idx outf_i;
-  const BlockDesc* blocks;   // non-null: scatter out_p into u_out (parameter layout)
+  const BlockDesc* blocks;   // non-null: scatter out_p into u_out (parameter layout); with
+                             // 128 x 256 tiles such an op may have no Cin
   float* u_out;
   float* unorm;              // per-problem sum of squares of the scattered out_p
 };

@@ -86,22 +86,34 @@ struct Bars {
   uint64_t full[kStages], empty[kStages];
   uint64_t acc_full[kRing], acc_empty[kRing];
   uint64_t drain;
+  uint64_t stg_free;              // a tile's epilogue no longer uses operand stage 1
+  uint64_t cin_full[kAccWarps];   // a warp's Cin row segment has landed in its staging
   uint32_t tmem_slot;
   int abort;
 };
-// Epilogue staging: per accumulator warp two 2 KB buffers, each one 32 x 16
-// chunk of split output (both planes) or of fp32 output, written by the
-// warp in the TMA swizzle and stored with one tensor store.
-constexpr int kStageBufBytes = 2048;
+// Epilogue staging: an epilogue step covers 32 rows x 32 columns of a warp's
+// row segment, 4 KB as split fp16 (both planes) or fp32.  Each accumulator
+// warp owns one 4 KB buffer in a region of its own (the 32 KB after the
+// operand stages) and, while its epilogue runs, three more in operand stage
+// 1 (12 KB of its 96 KB): one buffer per step of its 128-column segment.
+// Stage 1 is free then: a tile's last K slab has been read from it (K
+// slabs alternate between the stages and every tile has an even number),
+// and the producer loads the next tile's second slab into it only after
+// every warp's epilogue has released it (stg_free).  The MMA cannot run
+// ahead meanwhile anyway: its other tensor-memory buffer still holds the
+// finished tile.
+constexpr int kStageBufBytes = 4096;
 constexpr int kStagingOff = kStages * kStageBytes;
-constexpr int kBarsOff = kStagingOff + kAccWarps * 2 * kStageBufBytes;
+constexpr int kBarsOff = kStagingOff + kAccWarps * kStageBufBytes;
+static_assert(kStages == 2 && kAccWarps * 3 * kStageBufBytes <= kStageBytes, "borrowed staging exceeds a stage");
 constexpr int kSmemBytes = kBarsOff + 1024 + static_cast<int>(sizeof(Bars)) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory exceeds the per-block limit");
 
-// Output tensor maps of a launch: split and fp32 outputs of op 0 and op 1
-// (encoded for the outputs an op has, unless it scatters).
+// Epilogue tensor maps of a launch, per op: split and fp32 outputs and Cin
+// (split or fp32), boxes of 32 rows x 32 columns (encoded for what an op
+// has; scattering ops read no Cin).
 struct OutMaps {
-  CUtensorMap split[2], f32[2];
+  CUtensorMap split[2], f32[2], cin[2];
 };
 
 // Tiles of one problem.  Symmetric launches take the 128 x 256 tiles that
@@ -164,57 +176,75 @@ __device__ __forceinline__ void prefetch_cin_l2(const GemmOp& g, int p, size_t B
   }
 }
 
-// Staging writes: lane l holds row l of a 32 x 16 chunk.  Split chunk:
-// plane k (hi, lo) at k * 1 KB, row l at 32 l, its two 16-byte halves
-// swapped when bit 2 of l is set (32-byte swizzle: address bit 4 ^= bit 7).
-// fp32 chunk: row l at 64 l, 16-byte quarter h at h ^ ((l >> 1) & 3)
-// (64-byte swizzle: bits 5:4 ^= bits 8:7).  Eight consecutive lanes cover
-// all 32 banks, so each 16-byte store takes the minimum four wavefronts.
-__device__ __forceinline__ void stage_split16(uint8_t* buf, int lane, const float* w, bool& bad) {
-  __half2 hi[8], lo[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    split_f16x2(w[2 * j], w[2 * j + 1], hi[j], lo[j]);
-    bad |= f16_overflows(w[2 * j]) || f16_overflows(w[2 * j + 1]);
-  }
-  const int x = (lane >> 2) & 1;
-  uint8_t* r = buf + lane * 32;
-  *reinterpret_cast<uint4*>(r + 16 * x) = *reinterpret_cast<const uint4*>(&hi[0]);
-  *reinterpret_cast<uint4*>(r + 16 * (x ^ 1)) = *reinterpret_cast<const uint4*>(&hi[4]);
-  *reinterpret_cast<uint4*>(r + 1024 + 16 * x) = *reinterpret_cast<const uint4*>(&lo[0]);
-  *reinterpret_cast<uint4*>(r + 1024 + 16 * (x ^ 1)) = *reinterpret_cast<const uint4*>(&lo[4]);
+// Staging layouts; lane l holds row l of a 32 x 32 step.
+// - Split (and split Cin): plane k (hi, lo) at k * 2 KB, row l at 64 l, its
+//   16-byte quarter h (columns 8h..8h+7) at h ^ ((l >> 1) & 3) (64-byte
+//   swizzle: address bits 5:4 ^= bits 8:7).
+// - fp32: row l at 128 l, its 16-byte eighth h (columns 4h..4h+3) at
+//   h ^ (l & 7) (128-byte swizzle: bits 6:4 ^= bits 9:7).
+// Eight consecutive lanes cover all 32 banks, so each 16-byte access takes
+// the minimum four wavefronts.  Buffers are 4 KB-aligned.
+__device__ __forceinline__ uint32_t split_slot(int lane, int plane, int h) {
+  return static_cast<uint32_t>(plane * 2048 + lane * 64 + ((h ^ ((lane >> 1) & 3)) << 4));
 }
 
-__device__ __forceinline__ void stage_f32x16(uint8_t* buf, int lane, const float* v) {
-  const int x = (lane >> 1) & 3;
-  uint8_t* r = buf + lane * 64;
+// v[0], v[1]: the step's two 16-column chunks (already times the split factor)
+__device__ __forceinline__ void stage_split32(uint8_t* buf, int lane, const float (*v)[16], bool& bad) {
 #pragma unroll
-  for (int h = 0; h < 4; ++h)
-    *reinterpret_cast<float4*>(r + 16 * (h ^ x)) = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
-}
-
-// A warp's two staging buffers take the two 16-column chunks of one epilogue
-// step; before they are rewritten, the tensor stores issued from them one
-// step earlier must have finished reading them.
-struct Staging {
-  uint8_t* base;
-  __device__ __forceinline__ uint8_t* acquire(int lane) const {
-    if (lane == 0) bulk_wait_read<0>();
-    __syncwarp();
-    return base;
-  }
-  // the warp's writes go out as two tensor stores, chunks at (c0, c1, c2)
-  // and (c0 + 16, c1, c2)
-  __device__ __forceinline__ void release(int lane, const CUtensorMap* map, int c0, int c1, int c2) const {
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_3d(map, base, c0, c1, c2);
-      tma_store_3d(map, base + kStageBufBytes, c0 + 16, c1, c2);
-      bulk_commit();
+  for (int c = 0; c < 2; ++c) {
+    __half2 hi[8], lo[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      split_f16x2(v[c][2 * j], v[c][2 * j + 1], hi[j], lo[j]);
+      bad |= f16_overflows(v[c][2 * j]) || f16_overflows(v[c][2 * j + 1]);
     }
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 0, 2 * c)) = *reinterpret_cast<const uint4*>(&hi[0]);
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 0, 2 * c + 1)) = *reinterpret_cast<const uint4*>(&hi[4]);
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 1, 2 * c)) = *reinterpret_cast<const uint4*>(&lo[0]);
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 1, 2 * c + 1)) = *reinterpret_cast<const uint4*>(&lo[4]);
   }
-};
+}
+
+__device__ __forceinline__ void stage_f32x32(uint8_t* buf, int lane, const float (*v)[16]) {
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const float* x = &v[h >> 2][4 * (h & 3)];
+    *reinterpret_cast<float4*>(buf + lane * 128 + ((h ^ (lane & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+}
+
+// Cin of chunk c (0, 1) of a step from a split staging buffer, joined to fp32
+__device__ __forceinline__ void read_cin_chunk(const uint8_t* buf, int lane, int c, float* cj) {
+  SplitChunk r;
+  r.h[0] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 0, 2 * c));
+  r.h[1] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 0, 2 * c + 1));
+  r.l[0] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 1, 2 * c));
+  r.l[1] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 1, 2 * c + 1));
+  join_chunk(r, cj);
+}
+
+// fp32 Cin of chunk c (0, 1) of a step from an fp32 staging buffer
+__device__ __forceinline__ void read_cin_f32_chunk(const uint8_t* buf, int lane, int c, float* cj) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 x = *reinterpret_cast<const float4*>(buf + lane * 128 + (((4 * c + i) ^ (lane & 7)) << 4));
+    cj[4 * i] = x.x;
+    cj[4 * i + 1] = x.y;
+    cj[4 * i + 2] = x.z;
+    cj[4 * i + 3] = x.w;
+  }
+}
+
+// The warp's writes to buf go out as one tensor store at (c0, c1, c2).
+__device__ __forceinline__ void store_step(int lane, const CUtensorMap* map, const uint8_t* buf, int c0, int c1,
+                                           int c2) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(map, buf, c0, c1, c2);
+    bulk_commit();
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -241,6 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->acc_empty[b], kAccWarps);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->stg_free, kAccWarps);
+    for (int w = 0; w < kAccWarps; ++w) mbar_init(&bars->cin_full[w], 1);
     bars->abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
@@ -264,8 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kProdWarp && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
       uint32_t sc = 0, s = 0, epar = 1;  // loads issued, stage, parity of the stage's next release
+      uint32_t fpar = 0;                 // parity of the next stg_free phase
       bool stop = args.skip_loads != 0;
       for (long long t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+        const bool after_epilogue = t != blockIdx.x;  // stage 1 holds the previous tile's epilogue staging
         int op, p, ti, tj;
         decode_wide(args, tpp, ntn, t, op, p, ti, tj);
         const GemmOp& g = args.op[op];
@@ -277,6 +311,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             gemm_fail_timeout(abort_flag, args.status);
             stop = true;
             break;
+          }
+          if (kb == 1 && after_epilogue) {  // slab 1 goes to stage 1 (nk is even)
+            if (!mbar_wait(&bars->stg_free, fpar, abort_flag)) {
+              gemm_fail_timeout(abort_flag, args.status);
+              stop = true;
+              break;
+            }
+            fpar ^= 1u;
           }
           uint8_t* st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
@@ -370,7 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t B = static_cast<size_t>(args.B);
     const size_t BB = B * B;
     uint32_t hb = 0, hpar = 0;  // ring buffer, its fill parities
-    const Staging stg{smem + kStagingOff + warp * 2 * kStageBufBytes};
+    uint32_t cpar = 0;          // parity of this warp's next Cin arrival
+    bool cin_pending = false;   // a Cin load of this warp has not been waited for
     bool ok = true;
     for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
       float S[kCols];
@@ -432,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
       // epilogue of this thread's row segment (128 columns) from the buffer
-      // holding the finished sums; the buffer is released afterwards
+      // holding the finished sums, in four steps of 32 columns
       const uint32_t src = tbase + lane_off + hb * kN;
       // symmetric launches: this 128-column block q of the tile row ti is
       // written if q >= ti, and mirrored if q > ti (q < ti comes from the
@@ -442,71 +485,108 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool mirror = args.sym && q > ti;
       GemmEpilogue ep;
       ep.init(g, p, B, BB);
-      const int row0 = ti * kM + quad * 32;  // first row of this warp's chunks
-      // each step takes two 16-column chunks (one tensor-memory wait, one
-      // staging round); Cin streams one step ahead of use (L2 hits by now;
-      // a deeper ring does not fit the accumulator warps' registers)
-      GemmEpilogue::CinRaw pre[2];
-      const bool cin = write && ep.has_cin();
-      if (cin) {
-        pre[0] = ep.load_cin(B, BB, row, cbase);
-        pre[1] = ep.load_cin(B, BB, row, cbase + 16);
-      }
-#pragma unroll 1
-      for (int c = 0; c < (write ? kCols / 16 : 0); c += 2) {  // pre[0..1] hold chunks c, c+1
-        const int col0 = cbase + c * 16;
-        float v[2][16];
-        tmem_ld_32x32b_x16(src + 16 * c, reinterpret_cast<uint32_t*>(v[0]));
-        tmem_ld_32x32b_x16(src + 16 * c + 16, reinterpret_cast<uint32_t*>(v[1]));
-        tmem_ld_wait_regs<32>(reinterpret_cast<uint32_t*>(v));
+      const int row0 = ti * kM + quad * 32;  // first row of this warp's steps
+      uint8_t* const own = smem + kStagingOff + warp * kStageBufBytes;
+      uint8_t* const borrowed = smem + kStageBytes + warp * 3 * kStageBufBytes;
+      bool released = false;  // tensor-memory buffer handed back to the MMA
+      if (write) {
+        // step k stages in its own buffer, into which its Cin (split or
+        // fp32) arrives by TMA first: no waits on earlier stores
+        const bool cin = !ep.scatter && ep.has_cin();
+        if (cin && lane == 0) {
+          mbar_arrive_expect_tx(&bars->cin_full[warp], 4 * kStageBufBytes);
+          const int zc = ep.cin ? 2 * gemm_at(g.cin_i, p) : gemm_at(g.cinf_i, p);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float cj[16];
-          if (cin) {
-            ep.join_cin(pre[h], cj);
-            if (c + 2 < kCols / 16) pre[h] = ep.load_cin(B, BB, row, col0 + 32 + 16 * h);
+          for (int k = 0; k < 4; ++k)
+            tma_load_3d(k == 0 ? own : borrowed + (k - 1) * kStageBufBytes, &om.cin[op], &bars->cin_full[warp],
+                        cbase + 32 * k, row0, zc);
+        }
+        cin_pending = cin;
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          const int col0 = cbase + 32 * k;
+          uint8_t* buf = k == 0 ? own : borrowed + (k - 1) * kStageBufBytes;
+          float v[2][16];
+          tmem_ld_32x32b_x16(src + 32 * k, reinterpret_cast<uint32_t*>(v[0]));
+          tmem_ld_32x32b_x16(src + 32 * k + 16, reinterpret_cast<uint32_t*>(v[1]));
+          tmem_ld_wait_regs<32>(reinterpret_cast<uint32_t*>(v));
+          if (k == 3) {  // every tensor-memory read of the tile is done
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
+            released = true;
           }
-          ep.apply(row, col0 + 16 * h, v[h], cj);
-        }
-        if (ep.scatter) {
-          ep.check_finite(v[0]);
-          ep.check_finite(v[1]);
-          ep.scatter_chunk(g, row, col0, v[0]);
-          ep.scatter_chunk(g, row, col0 + 16, v[1]);
-          continue;
-        }
-        // row-major outputs leave through the staging buffers (one tensor
-        // store per 32 x 16 chunk instead of 32 row segments per store
-        // instruction); the mirror's stores are already coalesced
-        if (ep.os) {
-          uint8_t* buf = stg.acquire(lane);
+          if (cin && k == 0) {
+            if (!mbar_wait_sleep(&bars->cin_full[warp], cpar, abort_flag)) {
+              ok = false;
+              break;
+            }
+            cpar ^= 1u;
+            cin_pending = false;
+          }
+          // each lane reads, and below rewrites, only its own row of buf
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float w[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) w[j] = v[h][j] * ep.ss;
-            stage_split16(buf + h * kStageBufBytes, lane, w, ep.bad);
+            float cj[16];
+            if (cin) {
+              if (ep.cin) read_cin_chunk(buf, lane, h, cj);
+              else read_cin_f32_chunk(buf, lane, h, cj);
+            }
+            ep.apply(row, col0 + 16 * h, v[h], cj);
           }
-          stg.release(lane, &om.split[op], col0, row0, 2 * gemm_at(g.out_i, p));
+          if (ep.scatter) {
+            ep.check_finite(v[0]);
+            ep.check_finite(v[1]);
+            ep.scatter_chunk(g, row, col0, v[0]);
+            ep.scatter_chunk(g, row, col0 + 16, v[1]);
+            continue;
+          }
+          if (ep.os) {
+            float w[2][16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) w[h][j] = v[h][j] * ep.ss;
+            stage_split32(buf, lane, w, ep.bad);
+            store_step(lane, &om.split[op], buf, col0, row0, 2 * gemm_at(g.out_i, p));
+          }
+          if (ep.of) {
+            ep.check_finite(v[0]);
+            ep.check_finite(v[1]);
+            if (ep.os) {  // the split store must have read buf first
+              if (lane == 0) bulk_wait_read<0>();
+              __syncwarp();
+            }
+            stage_f32x32(buf, lane, v);
+            store_step(lane, &om.f32[op], buf, col0, row0, gemm_at(g.outf_i, p));
+          }
+          if (mirror) {
+            ep.store_mirror(B, BB, row, col0, v[0]);
+            ep.store_mirror(B, BB, row, col0 + 16, v[1]);
+          }
         }
-        if (ep.of) {
-          ep.check_finite(v[0]);
-          ep.check_finite(v[1]);
-          uint8_t* buf = stg.acquire(lane);
-          stage_f32x16(buf, lane, v[0]);
-          stage_f32x16(buf + kStageBufBytes, lane, v[1]);
-          stg.release(lane, &om.f32[op], col0, row0, gemm_at(g.outf_i, p));
-        }
-        if (mirror) {
-          ep.store_mirror(B, BB, row, col0, v[0]);
-          ep.store_mirror(B, BB, row, col0 + 16, v[1]);
+        if (!ok) {
+          if (lane == 0) gemm_fail_timeout(abort_flag, args.status);
+          break;
         }
       }
       ep.finish(g, p, args.status);
-      tc_fence_before();
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
+      }
+      // the staging buffers (own, and the borrowed part of stage 1) are
+      // free once this warp's stores have read them
+      if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
+      if (lane == 0) mbar_arrive(&bars->stg_free);
       hb ^= 1u;
+    }
+    // a Cin load still in flight after an abort lands before the CTA exits
+    if (cin_pending && lane == 0) {
+      volatile int never = 0;
+      mbar_wait(&bars->cin_full[warp], cpar, &never);
     }
     // this warp's tensor stores complete before the CTA's shared memory goes
     if (lane == 0) bulk_wait_all();
@@ -559,18 +639,30 @@ cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long lo
   // executed tensor-core flops: each 128 x 256 tile is one 2*128*256*B
   // product, done as three fp16 products
   const double flops = 3.0 * 2.0 * kM * kN * static_cast<double>(a.B) * static_cast<double>(total);
-  // output maps over the matrices the launch's problems write
+  // epilogue maps over the matrices the launch's problems write and read
   OutMaps om;
   std::memset(&om, 0, sizeof(om));
   for (int o = 0; o < a.nops; ++o) {
     const GemmOp& g = a.op[o];
-    if (g.nprob <= 0 || g.blocks) continue;
+    if (g.nprob <= 0) continue;
+    if (g.blocks) {  // a scattering op writes from registers and reads no Cin here
+      if (g.cin_split || g.cin_f32) return cudaErrorInvalidValue;
+      continue;
+    }
     if (g.out_split) {
       e = encode_epilogue_map(&om.split[o], g.out_split, false, a.B, 2 * idx_extent(g.out_i, g.nprob));
       if (e != cudaSuccess) return e;
     }
     if (g.out_f32) {
       e = encode_epilogue_map(&om.f32[o], g.out_f32, true, a.B, idx_extent(g.outf_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    }
+    if (g.cin_split) {
+      e = encode_epilogue_map(&om.cin[o], const_cast<__half*>(g.cin_split), false, a.B,
+                              2 * idx_extent(g.cin_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    } else if (g.cin_f32) {
+      e = encode_epilogue_map(&om.cin[o], const_cast<float*>(g.cin_f32), true, a.B, idx_extent(g.cinf_i, g.nprob));
       if (e != cudaSuccess) return e;
     }
   }

@@ -52,11 +52,11 @@ cudaError_t encode_epilogue_map(CUtensorMap* map, void* base, bool f32, int B, l
   const cuuint64_t esz = f32 ? 4u : 2u;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(B), static_cast<cuuint64_t>(B), static_cast<cuuint64_t>(depth)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(B) * esz, static_cast<cuuint64_t>(B) * B * esz};
-  cuuint32_t box[3] = {16u, 32u, f32 ? 1u : 2u};
+  cuuint32_t box[3] = {32u, 32u, f32 ? 1u : 2u};
   cuuint32_t estride[3] = {1u, 1u, 1u};
   CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims,
                    strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   f32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

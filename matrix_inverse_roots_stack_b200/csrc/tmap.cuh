@@ -20,11 +20,11 @@ cudaError_t encode_f16_3d_map(CUtensorMap* map, const void* base, int cols, int 
 // 128-byte swizzle.  Returns cudaSuccess or cudaErrorInvalidValue.
 cudaError_t encode_split_stack_map(CUtensorMap* map, const void* base, int B, int nmat, int box_rows = 128);
 
-// Encode a 3-D tiled map for epilogue chunks of a stack of B x B matrices:
-// split fp16 (f32 = false: dims {B, B, depth = 2 * nmat}, box {16, 32, 2},
-// both planes of a 32 x 16 chunk, 32-byte swizzle) or fp32 (dims {B, B,
-// depth = nmat}, box {16, 32, 1}, 64-byte swizzle).  base must be 16-byte
-// aligned.  Returns cudaSuccess or cudaErrorInvalidValue.
+// Encode a 3-D tiled map for 32 x 32 epilogue steps of a stack of B x B
+// matrices: split fp16 (f32 = false: dims {B, B, depth = 2 * nmat}, box
+// {32, 32, 2}, both planes, 64-byte swizzle) or fp32 (dims {B, B, depth =
+// nmat}, box {32, 32, 1}, 128-byte swizzle).  base must be 16-byte aligned.
+// Returns cudaSuccess or cudaErrorInvalidValue.
 cudaError_t encode_epilogue_map(CUtensorMap* map, void* base, bool f32, int B, long long depth);
 
 }  // namespace dash

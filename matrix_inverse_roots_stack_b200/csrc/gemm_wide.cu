@@ -87,7 +87,8 @@ struct Bars {
   uint64_t acc_full[kRing], acc_empty[kRing];
   uint64_t drain;
   uint64_t stg_free;              // a tile's epilogue no longer uses operand stage 1
-  uint64_t cin_full[kAccWarps];   // a warp's Cin row segment has landed in its staging
+  uint64_t cin0_full[kAccWarps];  // Cin of a warp's first epilogue step has landed in its own buffer
+  uint64_t cin_full[kAccWarps];   // Cin of its other three steps has landed in stage 1
   uint32_t tmem_slot;
   int abort;
 };
@@ -272,7 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->stg_free, kAccWarps);
-    for (int w = 0; w < kAccWarps; ++w) mbar_init(&bars->cin_full[w], 1);
+    for (int w = 0; w < kAccWarps; ++w) {
+      mbar_init(&bars->cin0_full[w], 1);
+      mbar_init(&bars->cin_full[w], 1);
+    }
     bars->abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
@@ -412,8 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t B = static_cast<size_t>(args.B);
     const size_t BB = B * B;
     uint32_t hb = 0, hpar = 0;  // ring buffer, its fill parities
-    uint32_t cpar = 0;          // parity of this warp's next Cin arrival
-    bool cin_pending = false;   // a Cin load of this warp has not been waited for
+    uint32_t cpar = 0;          // parity of this warp's next Cin arrivals (both barriers)
+    bool cin0_pending = false;  // a Cin load of this warp has not been waited for (own buffer,
+    bool cin_pending = false;   // stage 1)
     bool ok = true;
     for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
       float S[kCols];
@@ -430,8 +435,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pf_fill = nk > kPrefetchSlabs ? (nk - kPrefetchSlabs) * kFills : 0;
       // fill sg of the tile: S += its product (the last fill's sums go back
       // into its buffer for the epilogue instead of releasing it)
+      // the epilogue's first step takes its Cin from the warp's own buffer
+      // (free since the previous epilogue), loaded while the last slabs run
+      const int q = 2 * tj + cgrp;
+      const bool write = !args.sym || q >= ti;
+      const bool cin = write && !g.blocks && (g.cin_split || g.cin_f32);
+      uint8_t* const own = smem + kStagingOff + warp * kStageBufBytes;
+      uint8_t* const borrowed = smem + kStageBytes + warp * 3 * kStageBufBytes;
+      const int row0 = ti * kM + quad * 32;  // first row of this warp's steps
+      const int zc = g.cin_split ? 2 * gemm_at(g.cin_i, p) : gemm_at(g.cinf_i, p);
       for (int sg = 0; sg < nfill; ++sg) {
-        if (sg == pf_fill) prefetch_cin_l2(g, p, B, BB, row, cbase);
+        if (sg == pf_fill) {
+          prefetch_cin_l2(g, p, B, BB, row, cbase);
+          if (cin) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&bars->cin0_full[warp], kStageBufBytes);
+              tma_load_3d(own, &om.cin[op], &bars->cin0_full[warp], cbase, row0, zc);
+            }
+            cin0_pending = true;
+          }
+        }
         // waiting warps sleep in the barrier, leaving the issue slots of
         // their scheduler to the MMA and TMA threads
         if (!mbar_wait_sleep(&bars->acc_full[hb], (hpar >> hb) & 1u, abort_flag)) {
@@ -480,28 +503,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       // symmetric launches: this 128-column block q of the tile row ti is
       // written if q >= ti, and mirrored if q > ti (q < ti comes from the
       // mirror of block (q, ti))
-      const int q = 2 * tj + cgrp;
-      const bool write = !args.sym || q >= ti;
       const bool mirror = args.sym && q > ti;
       GemmEpilogue ep;
       ep.init(g, p, B, BB);
-      const int row0 = ti * kM + quad * 32;  // first row of this warp's steps
-      uint8_t* const own = smem + kStagingOff + warp * kStageBufBytes;
-      uint8_t* const borrowed = smem + kStageBytes + warp * 3 * kStageBufBytes;
       bool released = false;  // tensor-memory buffer handed back to the MMA
       if (write) {
         // step k stages in its own buffer, into which its Cin (split or
-        // fp32) arrives by TMA first: no waits on earlier stores
-        const bool cin = !ep.scatter && ep.has_cin();
-        if (cin && lane == 0) {
-          mbar_arrive_expect_tx(&bars->cin_full[warp], 4 * kStageBufBytes);
-          const int zc = ep.cin ? 2 * gemm_at(g.cin_i, p) : gemm_at(g.cinf_i, p);
+        // fp32) arrives by TMA first: no waits on earlier stores.  Steps
+        // 1-3 use stage 1, free now that the tile's MMAs are done.
+        if (cin) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bars->cin_full[warp], 3 * kStageBufBytes);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tma_load_3d(k == 0 ? own : borrowed + (k - 1) * kStageBufBytes, &om.cin[op], &bars->cin_full[warp],
-                        cbase + 32 * k, row0, zc);
+            for (int k = 1; k < 4; ++k)
+              tma_load_3d(borrowed + (k - 1) * kStageBufBytes, &om.cin[op], &bars->cin_full[warp], cbase + 32 * k,
+                          row0, zc);
+          }
+          cin_pending = true;
         }
-        cin_pending = cin;
 #pragma unroll 1
         for (int k = 0; k < 4; ++k) {
           const int col0 = cbase + 32 * k;
@@ -516,13 +535,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
             released = true;
           }
-          if (cin && k == 0) {
-            if (!mbar_wait_sleep(&bars->cin_full[warp], cpar, abort_flag)) {
+          if (cin && k < 2) {
+            if (!mbar_wait_sleep(k == 0 ? &bars->cin0_full[warp] : &bars->cin_full[warp], cpar, abort_flag)) {
               ok = false;
               break;
             }
-            cpar ^= 1u;
-            cin_pending = false;
+            if (k == 0) {
+              cin0_pending = false;
+            } else {
+              cpar ^= 1u;
+              cin_pending = false;
+            }
           }
           // each lane reads, and below rewrites, only its own row of buf
 #pragma unroll
@@ -584,9 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       hb ^= 1u;
     }
     // a Cin load still in flight after an abort lands before the CTA exits
-    if (cin_pending && lane == 0) {
+    if (lane == 0) {
       volatile int never = 0;
-      mbar_wait(&bars->cin_full[warp], cpar, &never);
+      if (cin0_pending) mbar_wait(&bars->cin0_full[warp], cpar, &never);
+      if (cin_pending) mbar_wait(&bars->cin_full[warp], cpar, &never);
     }
     // this warp's tensor stores complete before the CTA's shared memory goes
     if (lane == 0) bulk_wait_all();

@@ -1,6 +1,7 @@
 // Batched split-fp16 GEMM with 128 x 256 output tiles (sm_100a), for
-// launches whose block size is a multiple of 256 (split-fp16 products;
-// symmetric launches take the tiles that reach the upper triangle).
+// launches whose block size is a multiple of 256 (split-fp16 products, or
+// single-pass fp16 products for the fp16 coupled Newton; symmetric launches
+// take the tiles that reach the upper triangle).
 //
 // Split-fp16 products as in gemm.cu (hi*lo + lo*hi into a fresh
 // tensor-memory buffer, then hi*hi with that buffer scaled by 2^-11), with a
@@ -67,9 +68,6 @@ constexpr int kBBytes = kN * kKBlk * 2;                // 32 KB per plane and sl
 constexpr int kStageBytes = 2 * kABytes + 2 * kBBytes;  // A hi, A lo, B hi, B lo
 constexpr int kStages = 2;
 constexpr int kRing = 2;                               // product buffers of kN columns
-constexpr int kFillSteps = 2;                          // K=16 steps a buffer takes before its flush
-constexpr int kFills = kKBlk / 16 / kFillSteps;        // buffer fills per K slab
-static_assert(kFills * kFillSteps * 16 == kKBlk, "fills must tile the K slab");
 constexpr int kChunk = 32;                             // columns per tensor-memory load batch of a flush
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAccWarps = 8;                           // warps 0-7
@@ -247,10 +245,17 @@ __device__ __forceinline__ void store_step(int lane, const CUtensorMap* map, con
   }
 }
 
+// kSingle: single-pass fp16 products (hi planes only, one MMA per K=16
+// step, a whole K slab per buffer; the fp16 coupled-Newton mode); otherwise
+// split-fp16 products with two K=16 steps per buffer.
+template <bool kSingle>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                      const __grid_constant__ OutMaps om, const GemmArgs args, const long long total) {
+  constexpr int kFillSteps = kSingle ? 4 : 2;          // K=16 steps a buffer takes before its flush
+  constexpr int kFills = kKBlk / 16 / kFillSteps;      // buffer fills per K slab
+  static_assert(kFills * kFillSteps * 16 == kKBlk, "fills must tile the K slab");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -325,11 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             fpar ^= 1u;
           }
           uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
+          mbar_arrive_expect_tx(&bars->full[s], kSingle ? kABytes + kBBytes : kStageBytes);
           tma_load_3d(st, ta, &bars->full[s], kb * kKBlk, ti * kM, 2 * am);
-          tma_load_3d(st + kABytes, ta, &bars->full[s], kb * kKBlk, ti * kM, 2 * am + 1);
+          if (!kSingle) tma_load_3d(st + kABytes, ta, &bars->full[s], kb * kKBlk, ti * kM, 2 * am + 1);
 #pragma unroll
-          for (int pl = 0; pl < 2; ++pl) {
+          for (int pl = 0; pl < (kSingle ? 1 : 2); ++pl) {
             uint8_t* dst = st + 2 * kABytes + pl * kBBytes;
             if (g.b_mn) {  // rows kb*64.. of B, columns tj*256.. as four 64-column boxes
 #pragma unroll
@@ -379,17 +384,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t d = tbase + hb * kN;
             const int k0 = f * kFillSteps;
-            // cross terms hi*lo + lo*hi of the fill's K=16 steps into a fresh
-            // buffer, then hi*hi of its first step plus 2^-11 times that sum,
-            // then hi*hi of its other steps
+            if (kSingle) {  // hi*hi of the slab's four steps into a fresh buffer
 #pragma unroll
-            for (int kk = k0; kk < k0 + kFillSteps; ++kk) {
-              mma_f16_ss(d, ah + 2u * kk, bl + bstep * kk, idesc, kk > k0 ? 1u : 0u);
-              mma_f16_ss(d, al + 2u * kk, bh + bstep * kk, idesc, 1u);
+              for (int kk = k0; kk < k0 + kFillSteps; ++kk)
+                mma_f16_ss(d, ah + 2u * kk, bh + bstep * kk, idesc, kk > k0 ? 1u : 0u);
+            } else {
+              // cross terms hi*lo + lo*hi of the fill's K=16 steps into a
+              // fresh buffer, then hi*hi of its first step plus 2^-11 times
+              // that sum, then hi*hi of its other steps
+#pragma unroll
+              for (int kk = k0; kk < k0 + kFillSteps; ++kk) {
+                mma_f16_ss(d, ah + 2u * kk, bl + bstep * kk, idesc, kk > k0 ? 1u : 0u);
+                mma_f16_ss(d, al + 2u * kk, bh + bstep * kk, idesc, 1u);
+              }
+              mma_f16_ss_acc_down11(d, ah + 2u * k0, bh + bstep * k0, idesc);
+#pragma unroll
+              for (int kk = k0 + 1; kk < k0 + kFillSteps; ++kk)
+                mma_f16_ss(d, ah + 2u * kk, bh + bstep * kk, idesc, 1u);
             }
-            mma_f16_ss_acc_down11(d, ah + 2u * k0, bh + bstep * k0, idesc);
-#pragma unroll
-            for (int kk = k0 + 1; kk < k0 + kFillSteps; ++kk) mma_f16_ss(d, ah + 2u * kk, bh + bstep * kk, idesc, 1u);
             mma_commit(&bars->acc_full[hb]);
             hb ^= 1u;
           }
@@ -624,13 +636,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Registers a thread of gemm_wide_kernel was compiled with (once per process).
+// Registers a thread of gemm_wide_kernel was compiled with (once per
+// process): the count both instantiations share, or 0 if they differ.
 int wide_kernel_regs() {
   static std::atomic<int> regs{-1};
   int r = regs.load();
   if (r < 0) {
-    cudaFuncAttributes fa;
-    r = cudaFuncGetAttributes(&fa, gemm_wide_kernel) == cudaSuccess ? fa.numRegs : 0;
+    cudaFuncAttributes f0, f1;
+    const bool ok = cudaFuncGetAttributes(&f0, gemm_wide_kernel<false>) == cudaSuccess &&
+                    cudaFuncGetAttributes(&f1, gemm_wide_kernel<true>) == cudaSuccess;
+    r = ok && f0.numRegs == f1.numRegs ? f0.numRegs : 0;
     regs.store(r);
   }
   return r;
@@ -647,22 +662,29 @@ long long idx_extent(const Idx& i, int nprob) {
 }  // namespace
 
 bool gemm_wide_supported(const GemmArgs& a) {
-  // the register split needs the launch to hold exactly kLaunchRegs a thread
-  return a.single_pass == 0 && a.B % kN == 0 && a.B >= kN && wide_kernel_regs() == kLaunchRegs;
+  // the register split needs the launch to hold exactly kLaunchRegs a thread.
+  // Single-pass products at B = 256 stay on 128 x 128 tiles: their buffers
+  // hold one MMA's work per flush, and 128 x 256 tiles cannot skip any of a
+  // symmetric launch's lower triangle (3.66 against 3.50 ms for 256 fp16
+  // coupled-Newton roots of 256).
+  if (a.single_pass && a.B < 512) return false;
+  return a.B % kN == 0 && a.B >= kN && wide_kernel_regs() == kLaunchRegs;
 }
 
 int gemm_wide_regs() { return wide_kernel_regs(); }
 
 cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long long nprob, cudaStream_t stream) {
-  static std::atomic<unsigned long long> attr_set;
-  cudaError_t e = smem_limit_once(gemm_wide_kernel, kSmemBytes, attr_set);
+  auto kern = a.single_pass ? gemm_wide_kernel<true> : gemm_wide_kernel<false>;
+  static std::atomic<unsigned long long> attr_set[2];
+  cudaError_t e = smem_limit_once(kern, kSmemBytes, attr_set[a.single_pass ? 1 : 0]);
   if (e != cudaSuccess) return e;
   const long long total = static_cast<long long>(wide_tiles_per_problem(a.B, a.sym)) * nprob;
   const long long sms = gemm_sm_count();
   const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
   // executed tensor-core flops: each 128 x 256 tile is one 2*128*256*B
-  // product, done as three fp16 products
-  const double flops = 3.0 * 2.0 * kM * kN * static_cast<double>(a.B) * static_cast<double>(total);
+  // product, done as three fp16 products (one in single-pass mode)
+  const double flops =
+      (a.single_pass ? 1.0 : 3.0) * 2.0 * kM * kN * static_cast<double>(a.B) * static_cast<double>(total);
   // epilogue maps over the matrices the launch's problems write and read
   OutMaps om;
   std::memset(&om, 0, sizeof(om));
@@ -691,7 +713,7 @@ cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long lo
     }
   }
   const int slot = prof_begin(kProfGemmWide, stream, flops);
-  gemm_wide_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], om, a, total);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], om, a, total);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

@@ -217,6 +217,16 @@ def test_coupled_newton_fp16(torch, kappa, iters, tol):
         assert rel(X[i], r) < tol, (i, rel(X[i], r))
 
 
+def test_coupled_newton_fp16_block_512(torch):
+    # the same single-pass products at B=512, where they run on 128 x 256
+    # tiles (a whole K slab per tensor-memory buffer); bound as at B=256
+    A = workloads.spd_stack_geometric(3, 512, 1e2, seed=3)
+    X, lam, rc = gpu_cn(torch, A, 12, True)
+    assert rc == 0
+    for i, r in enumerate(cn_level2(A, 0.0, lam, 12)):
+        assert rel(X[i], r) < 3e-3, (i, rel(X[i], r))
+
+
 def test_coupled_newton_fp16_reports_divergence(torch):
     # at kappa=1e6 fp16 rounding pushes small eigenvalues of M below zero and
     # the iteration diverges; the status word says so instead of returning

@@ -140,11 +140,13 @@ def test_standalone_workload_full_size(torch):
     assert max(errs) < ROOT_TOL, max(errs)
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(torch):
+@pytest.mark.parametrize("B", [128, 256])
+def test_bounded_wait_reports_timeout_and_context_survives(torch, B):
     # a GEMM launch that never receives its operand tiles: every wait gives up
     # after its limit, the status word says TIMEOUT, and the next call works
+    # (B=128: 128 x 128 tiles; B=256: 128 x 256 tiles)
     from matrix_inverse_roots_stack_b200 import binding as bd
-    A = workloads.spd_stack_geometric(1, 128, 10.0, seed=12)
+    A = workloads.spd_stack_geometric(1, B, 10.0, seed=12)
     lib = bd.load()
     assert lib.shampoo_debug_inject_timeout() == 0
     X, lam, rc, _ = gpu_roots(torch, A, "ndb", iters1=2, iters2=2)

@@ -57,7 +57,15 @@ struct Bars {
   uint32_t tmem_slot;
   int abort;
 };
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + static_cast<int>(sizeof(Bars)) + 64;
+// Output staging: per output warp two 4 KB buffers, each one 32 x 32 step of
+// split fp16 (both planes) or fp32 output in the TMA swizzle, stored with one
+// tensor store; a buffer is rewritten once the store from it two steps ago
+// has read it.
+constexpr int kStageBufBytes = 4096;
+constexpr int kStagingOff = kStages * kStageBytes;
+constexpr int kBarsOff = kStagingOff + kOutWarps * 2 * kStageBufBytes;
+constexpr int kSmemBytes = kBarsOff + 1024 + static_cast<int>(sizeof(Bars)) + 64;
+static_assert(kSmemBytes <= 232448, "shared memory exceeds the per-block limit");
 
 // Tile t of a problem -> (tile row, tile column).  sym: upper triangle of
 // the nt x nt square tile grid only, enumerated row by row.
@@ -102,11 +110,11 @@ template <bool kSingle>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_split_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                       const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                      const GemmArgs args, const long long total) {
+                      const __grid_constant__ OutMaps om, const GemmArgs args, const long long total) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  Bars* bars = reinterpret_cast<Bars*>(smem + kBarsOff);
   volatile int* abort_flag = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -315,6 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t B = static_cast<size_t>(args.B);
     const size_t BB = B * B;
     uint32_t ppar = 0;
+    uint8_t* const stg = smem + kStagingOff + (warp - kOutWarp0) * 2 * kStageBufBytes;
+    int nb = 0;  // next staging buffer
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
       int op, p, ti, tj;
       decode(args, tpp, nt, t, op, p, ti, tj);
@@ -324,34 +334,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool mirror = args.sym && (ti != tj);
       GemmEpilogue ep;
       ep.init(g, p, B, BB);
-      GemmEpilogue::CinRaw nxt;  // Cin is loaded one chunk ahead, the first before the wait
-      if (ep.has_cin()) nxt = ep.load_cin(B, BB, row, cbase);
+      const bool cin = ep.has_cin();
+      const int row0 = ti * kTile + quad * 32;  // first row of this warp's steps
       if (!mbar_wait_sleep(&bars->park_full, ppar, abort_flag)) {
         if (threadIdx.x == kOutWarp0 * 32) gemm_fail_timeout(abort_flag, args.status);
         break;
       }
       ppar ^= 1u;
       tc_fence_after();
+      // four steps of 32 columns; row-major outputs leave through the
+      // staging buffers (a store instruction whose 32 lanes each write a
+      // different row would touch 32 lines), the mirror's stores are
+      // already coalesced, scattered outputs go straight to the parameters
 #pragma unroll 1
-      for (int c = 0; c < kTile / 16; ++c) {
-        const int col0 = cbase + c * 16;
-        float v[16], cj[16];
-        tmem_ld_32x32b_x16(tbase + lane_off + kColPark + 16 * c, reinterpret_cast<uint32_t*>(v));
-        tmem_ld_wait_regs<16>(reinterpret_cast<uint32_t*>(v));
-        if (c + 1 == kTile / 16) {  // the park buffer is free for the next tile
+      for (int k = 0; k < kTile / 32; ++k) {
+        const int col0 = cbase + 32 * k;
+        GemmEpilogue::CinRaw pre[2];  // in flight during the tensor-memory loads
+        if (cin) {
+          pre[0] = ep.load_cin(B, BB, row, col0);
+          pre[1] = ep.load_cin(B, BB, row, col0 + 16);
+        }
+        float v[2][16];
+        tmem_ld_32x32b_x16(tbase + lane_off + kColPark + 32 * k, reinterpret_cast<uint32_t*>(v[0]));
+        tmem_ld_32x32b_x16(tbase + lane_off + kColPark + 32 * k + 16, reinterpret_cast<uint32_t*>(v[1]));
+        tmem_ld_wait_regs<32>(reinterpret_cast<uint32_t*>(v));
+        if (k + 1 == kTile / 32) {  // the park buffer is free for the next tile
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->park_empty);
         }
-        if (ep.has_cin()) {
-          const GemmEpilogue::CinRaw cur = nxt;
-          if (c + 1 < kTile / 16) nxt = ep.load_cin(B, BB, row, col0 + 16);
-          ep.join_cin(cur, cj);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float cj[16];
+          if (cin) ep.join_cin(pre[h], cj);
+          ep.apply(row, col0 + 16 * h, v[h], cj);
         }
-        ep.chunk(g, B, BB, row, col0, v, cj, mirror);
+        if (ep.scatter) {  // through fp32 staging: lane l writes column l, row by row
+          ep.check_finite(v[0]);
+          ep.check_finite(v[1]);
+          uint8_t* buf = stg + nb * kStageBufBytes;
+          __syncwarp();
+          stage_f32x32(buf, lane, v);
+          __syncwarp();
+          scatter_step(buf, lane, g, ep.bd, row0, col0, ep.sumsq);
+          nb ^= 1;
+          continue;
+        }
+        if (mirror) {
+          ep.store_mirror(B, BB, row, col0, v[0]);
+          ep.store_mirror(B, BB, row, col0 + 16, v[1]);
+        }
+        if (ep.of) {
+          ep.check_finite(v[0]);
+          ep.check_finite(v[1]);
+          uint8_t* buf = stg + nb * kStageBufBytes;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          stage_f32x32(buf, lane, v);
+          store_step(lane, &om.f32[op], buf, col0, row0, gemm_at(g.outf_i, p));
+          nb ^= 1;
+        }
+        if (ep.os) {  // split output, scaled in place
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[h][j] *= ep.ss;
+          uint8_t* buf = stg + nb * kStageBufBytes;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          stage_split32(buf, lane, v, ep.bad);
+          store_step(lane, &om.split[op], buf, col0, row0, 2 * gemm_at(g.out_i, p));
+          nb ^= 1;
+        }
       }
       ep.finish(g, p, args.status);
     }
+    // this warp's tensor stores complete before the CTA's shared memory goes
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -391,8 +450,11 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
     if (e != cudaSuccess) return e;
   }
   if (wide) return launch_gemm_wide(maps, a, nprob, stream);
-  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const GemmArgs,
-               const long long) = a.single_pass ? gemm_split_kernel<true> : gemm_split_kernel<false>;
+  OutMaps om;
+  cudaError_t me = encode_out_maps(a, &om);
+  if (me != cudaSuccess) return me;
+  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const OutMaps,
+               const GemmArgs, const long long) = a.single_pass ? gemm_split_kernel<true> : gemm_split_kernel<false>;
   static std::atomic<unsigned long long> attr_set[2];
   cudaError_t e = smem_limit_once(kern, kSmemBytes, attr_set[a.single_pass ? 1 : 0]);
   if (e != cudaSuccess) return e;
@@ -406,7 +468,7 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   const double flops = (a.single_pass ? 1.0 : 3.0) * 2.0 * kTile * kTile * static_cast<double>(a.B) *
                        static_cast<double>(total);
   const int slot = prof_begin(kProfGemm, stream, flops);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], a, total);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], om, a, total);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

@@ -286,6 +286,107 @@ struct GemmEpilogue {
   }
 };
 
+// Epilogue tensor maps of a launch, per op: split and fp32 outputs and Cin
+// (split or fp32), boxes of 32 rows x 32 columns (encoded for what an op
+// has; scattering ops read no Cin).
+struct OutMaps {
+  CUtensorMap split[2], f32[2], cin[2];
+};
+
+// Staging layouts; lane l holds row l of a 32 x 32 step.
+// - Split (and split Cin): plane k (hi, lo) at k * 2 KB, row l at 64 l, its
+//   16-byte quarter h (columns 8h..8h+7) at h ^ ((l >> 1) & 3) (64-byte
+//   swizzle: address bits 5:4 ^= bits 8:7).
+// - fp32: row l at 128 l, its 16-byte eighth h (columns 4h..4h+3) at
+//   h ^ (l & 7) (128-byte swizzle: bits 6:4 ^= bits 9:7).
+// Eight consecutive lanes cover all 32 banks, so each 16-byte access takes
+// the minimum four wavefronts.  Buffers are 4 KB-aligned.
+__device__ __forceinline__ uint32_t split_slot(int lane, int plane, int h) {
+  return static_cast<uint32_t>(plane * 2048 + lane * 64 + ((h ^ ((lane >> 1) & 3)) << 4));
+}
+
+// v[0], v[1]: the step's two 16-column chunks (already times the split factor)
+__device__ __forceinline__ void stage_split32(uint8_t* buf, int lane, const float (*v)[16], bool& bad) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    __half2 hi[8], lo[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      split_f16x2(v[c][2 * j], v[c][2 * j + 1], hi[j], lo[j]);
+      bad |= f16_overflows(v[c][2 * j]) || f16_overflows(v[c][2 * j + 1]);
+    }
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 0, 2 * c)) = *reinterpret_cast<const uint4*>(&hi[0]);
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 0, 2 * c + 1)) = *reinterpret_cast<const uint4*>(&hi[4]);
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 1, 2 * c)) = *reinterpret_cast<const uint4*>(&lo[0]);
+    *reinterpret_cast<uint4*>(buf + split_slot(lane, 1, 2 * c + 1)) = *reinterpret_cast<const uint4*>(&lo[4]);
+  }
+}
+
+__device__ __forceinline__ void stage_f32x32(uint8_t* buf, int lane, const float (*v)[16]) {
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const float* x = &v[h >> 2][4 * (h & 3)];
+    *reinterpret_cast<float4*>(buf + lane * 128 + ((h ^ (lane & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+}
+
+// Cin of chunk c (0, 1) of a step from a split staging buffer, joined to fp32
+__device__ __forceinline__ void read_cin_chunk(const uint8_t* buf, int lane, int c, float* cj) {
+  SplitChunk r;
+  r.h[0] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 0, 2 * c));
+  r.h[1] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 0, 2 * c + 1));
+  r.l[0] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 1, 2 * c));
+  r.l[1] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 1, 2 * c + 1));
+  join_chunk(r, cj);
+}
+
+// fp32 Cin of chunk c (0, 1) of a step from an fp32 staging buffer
+__device__ __forceinline__ void read_cin_f32_chunk(const uint8_t* buf, int lane, int c, float* cj) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 x = *reinterpret_cast<const float4*>(buf + lane * 128 + (((4 * c + i) ^ (lane & 7)) << 4));
+    cj[4 * i] = x.x;
+    cj[4 * i + 1] = x.y;
+    cj[4 * i + 2] = x.z;
+    cj[4 * i + 3] = x.w;
+  }
+}
+
+// The warp's writes to buf go out as one tensor store at (c0, c1, c2).
+__device__ __forceinline__ void store_step(int lane, const CUtensorMap* map, const uint8_t* buf, int c0, int c1,
+                                           int c2) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(map, buf, c0, c1, c2);
+    bulk_commit();
+  }
+}
+
+// kSingle: single-pass fp16 products (hi planes only, one MMA per K=16
+// step, a whole K slab per buffer; the fp16 coupled-Newton mode); otherwise
+// split-fp16 products with two K=16 steps per buffer.
+// A staged fp32 step (stage_f32x32) scattered into parameter layout: lane l
+// writes column col0 + l of rows row0.. (coalesced across the lanes), inside
+// the block's extent only, and adds its squares to sumsq.
+__device__ __forceinline__ void scatter_step(const uint8_t* buf, int lane, const GemmOp& g, const BlockDesc& bd,
+                                             int row0, int col0, float& sumsq) {
+  const int col = col0 + lane;
+  if (col >= bd.bc) return;
+  float* dst = g.u_out + bd.off + static_cast<long long>(bd.r0) * bd.pitch + bd.c0 + col;
+  const int nr = bd.br - row0 < 32 ? bd.br - row0 : 32;
+#pragma unroll 4
+  for (int r = 0; r < nr; ++r) {
+    const float x =
+        *reinterpret_cast<const float*>(buf + r * 128 + ((((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2)));
+    dst[static_cast<long long>(row0 + r) * bd.pitch] = x;
+    sumsq += x * x;
+  }
+}
+
+// The epilogue maps of a launch's ops (see OutMaps).
+cudaError_t encode_out_maps(const GemmArgs& a, OutMaps* om);
+
 int gemm_sm_count();
 
 // The 128 x 256 tile kernel (gemm_wide.cu): whether it takes a launch, and

@@ -108,12 +108,6 @@ static_assert(kStages == 2 && kAccWarps * 3 * kStageBufBytes <= kStageBytes, "bo
 constexpr int kSmemBytes = kBarsOff + 1024 + static_cast<int>(sizeof(Bars)) + 64;
 static_assert(kSmemBytes <= 232448, "shared memory exceeds the per-block limit");
 
-// Epilogue tensor maps of a launch, per op: split and fp32 outputs and Cin
-// (split or fp32), boxes of 32 rows x 32 columns (encoded for what an op
-// has; scattering ops read no Cin).
-struct OutMaps {
-  CUtensorMap split[2], f32[2], cin[2];
-};
 
 // Tiles of one problem.  Symmetric launches take the 128 x 256 tiles that
 // reach the upper triangle, 2 tj + 1 >= ti in 128-column units: row ti has
@@ -175,79 +169,6 @@ __device__ __forceinline__ void prefetch_cin_l2(const GemmOp& g, int p, size_t B
   }
 }
 
-// Staging layouts; lane l holds row l of a 32 x 32 step.
-// - Split (and split Cin): plane k (hi, lo) at k * 2 KB, row l at 64 l, its
-//   16-byte quarter h (columns 8h..8h+7) at h ^ ((l >> 1) & 3) (64-byte
-//   swizzle: address bits 5:4 ^= bits 8:7).
-// - fp32: row l at 128 l, its 16-byte eighth h (columns 4h..4h+3) at
-//   h ^ (l & 7) (128-byte swizzle: bits 6:4 ^= bits 9:7).
-// Eight consecutive lanes cover all 32 banks, so each 16-byte access takes
-// the minimum four wavefronts.  Buffers are 4 KB-aligned.
-__device__ __forceinline__ uint32_t split_slot(int lane, int plane, int h) {
-  return static_cast<uint32_t>(plane * 2048 + lane * 64 + ((h ^ ((lane >> 1) & 3)) << 4));
-}
-
-// v[0], v[1]: the step's two 16-column chunks (already times the split factor)
-__device__ __forceinline__ void stage_split32(uint8_t* buf, int lane, const float (*v)[16], bool& bad) {
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    __half2 hi[8], lo[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      split_f16x2(v[c][2 * j], v[c][2 * j + 1], hi[j], lo[j]);
-      bad |= f16_overflows(v[c][2 * j]) || f16_overflows(v[c][2 * j + 1]);
-    }
-    *reinterpret_cast<uint4*>(buf + split_slot(lane, 0, 2 * c)) = *reinterpret_cast<const uint4*>(&hi[0]);
-    *reinterpret_cast<uint4*>(buf + split_slot(lane, 0, 2 * c + 1)) = *reinterpret_cast<const uint4*>(&hi[4]);
-    *reinterpret_cast<uint4*>(buf + split_slot(lane, 1, 2 * c)) = *reinterpret_cast<const uint4*>(&lo[0]);
-    *reinterpret_cast<uint4*>(buf + split_slot(lane, 1, 2 * c + 1)) = *reinterpret_cast<const uint4*>(&lo[4]);
-  }
-}
-
-__device__ __forceinline__ void stage_f32x32(uint8_t* buf, int lane, const float (*v)[16]) {
-#pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    const float* x = &v[h >> 2][4 * (h & 3)];
-    *reinterpret_cast<float4*>(buf + lane * 128 + ((h ^ (lane & 7)) << 4)) = make_float4(x[0], x[1], x[2], x[3]);
-  }
-}
-
-// Cin of chunk c (0, 1) of a step from a split staging buffer, joined to fp32
-__device__ __forceinline__ void read_cin_chunk(const uint8_t* buf, int lane, int c, float* cj) {
-  SplitChunk r;
-  r.h[0] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 0, 2 * c));
-  r.h[1] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 0, 2 * c + 1));
-  r.l[0] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 1, 2 * c));
-  r.l[1] = *reinterpret_cast<const uint4*>(buf + split_slot(lane, 1, 2 * c + 1));
-  join_chunk(r, cj);
-}
-
-// fp32 Cin of chunk c (0, 1) of a step from an fp32 staging buffer
-__device__ __forceinline__ void read_cin_f32_chunk(const uint8_t* buf, int lane, int c, float* cj) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 x = *reinterpret_cast<const float4*>(buf + lane * 128 + (((4 * c + i) ^ (lane & 7)) << 4));
-    cj[4 * i] = x.x;
-    cj[4 * i + 1] = x.y;
-    cj[4 * i + 2] = x.z;
-    cj[4 * i + 3] = x.w;
-  }
-}
-
-// The warp's writes to buf go out as one tensor store at (c0, c1, c2).
-__device__ __forceinline__ void store_step(int lane, const CUtensorMap* map, const uint8_t* buf, int c0, int c1,
-                                           int c2) {
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_3d(map, buf, c0, c1, c2);
-    bulk_commit();
-  }
-}
-
-// kSingle: single-pass fp16 products (hi planes only, one MMA per K=16
-// step, a whole K slab per buffer; the fp16 coupled-Newton mode); otherwise
-// split-fp16 products with two K=16 steps per buffer.
 template <bool kSingle>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -661,6 +582,33 @@ long long idx_extent(const Idx& i, int nprob) {
 
 }  // namespace
 
+cudaError_t encode_out_maps(const GemmArgs& a, OutMaps* om) {
+  cudaError_t e = cudaSuccess;
+  // epilogue maps over the matrices the launch's problems write and read
+  std::memset(om, 0, sizeof(*om));
+  for (int o = 0; o < a.nops; ++o) {
+    const GemmOp& g = a.op[o];
+    if (g.nprob <= 0 || g.blocks) continue;  // a scattering op writes from registers
+    if (g.out_split) {
+      e = encode_epilogue_map(&om->split[o], g.out_split, false, a.B, 2 * idx_extent(g.out_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    }
+    if (g.out_f32) {
+      e = encode_epilogue_map(&om->f32[o], g.out_f32, true, a.B, idx_extent(g.outf_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    }
+    if (g.cin_split) {
+      e = encode_epilogue_map(&om->cin[o], const_cast<__half*>(g.cin_split), false, a.B,
+                              2 * idx_extent(g.cin_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    } else if (g.cin_f32) {
+      e = encode_epilogue_map(&om->cin[o], const_cast<float*>(g.cin_f32), true, a.B, idx_extent(g.cinf_i, g.nprob));
+      if (e != cudaSuccess) return e;
+    }
+  }
+  return cudaSuccess;
+}
+
 bool gemm_wide_supported(const GemmArgs& a) {
   // the register split needs the launch to hold exactly kLaunchRegs a thread.
   // Single-pass products at B = 256 stay on 128 x 128 tiles: their buffers
@@ -685,33 +633,11 @@ cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long lo
   // product, done as three fp16 products (one in single-pass mode)
   const double flops =
       (a.single_pass ? 1.0 : 3.0) * 2.0 * kM * kN * static_cast<double>(a.B) * static_cast<double>(total);
-  // epilogue maps over the matrices the launch's problems write and read
+  for (int o = 0; o < a.nops; ++o)  // a scattering op reads no Cin on 128 x 256 tiles
+    if (a.op[o].nprob > 0 && a.op[o].blocks && (a.op[o].cin_split || a.op[o].cin_f32)) return cudaErrorInvalidValue;
   OutMaps om;
-  std::memset(&om, 0, sizeof(om));
-  for (int o = 0; o < a.nops; ++o) {
-    const GemmOp& g = a.op[o];
-    if (g.nprob <= 0) continue;
-    if (g.blocks) {  // a scattering op writes from registers and reads no Cin here
-      if (g.cin_split || g.cin_f32) return cudaErrorInvalidValue;
-      continue;
-    }
-    if (g.out_split) {
-      e = encode_epilogue_map(&om.split[o], g.out_split, false, a.B, 2 * idx_extent(g.out_i, g.nprob));
-      if (e != cudaSuccess) return e;
-    }
-    if (g.out_f32) {
-      e = encode_epilogue_map(&om.f32[o], g.out_f32, true, a.B, idx_extent(g.outf_i, g.nprob));
-      if (e != cudaSuccess) return e;
-    }
-    if (g.cin_split) {
-      e = encode_epilogue_map(&om.cin[o], const_cast<__half*>(g.cin_split), false, a.B,
-                              2 * idx_extent(g.cin_i, g.nprob));
-      if (e != cudaSuccess) return e;
-    } else if (g.cin_f32) {
-      e = encode_epilogue_map(&om.cin[o], const_cast<float*>(g.cin_f32), true, a.B, idx_extent(g.cinf_i, g.nprob));
-      if (e != cudaSuccess) return e;
-    }
-  }
+  e = encode_out_maps(a, &om);
+  if (e != cudaSuccess) return e;
   const int slot = prof_begin(kProfGemmWide, stream, flops);
   kern<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], om, a, total);
   prof_end(slot, stream);

@@ -1,8 +1,9 @@
 // Pieces shared by the two split-fp16 GEMM kernels (gemm.cu: 128 x 128 tiles
 // with a parked output stage; gemm_wide.cu: 128 x 256 tiles written out by
 // the accumulator warps): problem indexing, the MN-major operand descriptor,
-// the split-fp16 load/store helpers and the epilogue of one output row
-// segment, out = s_p * (alpha * a_p * acc + beta * Cin + gamma * I).
+// the split-fp16 helpers, the epilogue arithmetic of one output row
+// segment, out = s_p * (alpha * a_p * acc + beta * Cin + gamma * I), and the
+// shared-memory staging of 32 x 32 output steps for TMA tensor stores.
 #pragma once
 
 #include <cuda.h>
@@ -36,21 +37,6 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
-__device__ __forceinline__ void store_split16(__half* base, size_t BB, size_t idx, const float* v, bool& bad) {
-  __half2 hi[8], lo[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    split_f16x2(v[2 * j], v[2 * j + 1], hi[j], lo[j]);
-    bad |= f16_overflows(v[2 * j]) || f16_overflows(v[2 * j + 1]);
-  }
-  uint4* dh = reinterpret_cast<uint4*>(base + idx);
-  uint4* dl = reinterpret_cast<uint4*>(base + BB + idx);
-  dh[0] = *reinterpret_cast<const uint4*>(&hi[0]);  // hi[0..3]: columns 0..7
-  dh[1] = *reinterpret_cast<const uint4*>(&hi[4]);  // hi[4..7]: columns 8..15
-  dl[0] = *reinterpret_cast<const uint4*>(&lo[0]);
-  dl[1] = *reinterpret_cast<const uint4*>(&lo[4]);
-}
-
 // out(col0 + j, row) = v[j]: for a fixed j the 32 lanes (consecutive rows)
 // write consecutive addresses.
 __device__ __forceinline__ void store_split16_t(__half* base, size_t B, size_t BB, int row, int col0, const float* v,
@@ -71,17 +57,6 @@ __device__ __forceinline__ void store_split16_t(__half* base, size_t B, size_t B
 struct SplitChunk {
   uint4 h[2], l[2];
 };
-
-__device__ __forceinline__ SplitChunk ld_chunk(const __half* base, size_t BB, size_t idx) {
-  SplitChunk c;
-  const uint4* h4 = reinterpret_cast<const uint4*>(base + idx);
-  const uint4* l4 = reinterpret_cast<const uint4*>(base + BB + idx);
-  c.h[0] = h4[0];
-  c.h[1] = h4[1];
-  c.l[0] = l4[0];
-  c.l[1] = l4[1];
-  return c;
-}
 
 __device__ __forceinline__ void join_chunk(const SplitChunk& c, float* out) {
 #pragma unroll
@@ -249,30 +224,6 @@ struct GemmEpilogue {
 #pragma unroll
       for (int j = 0; j < 16; ++j) of[(col0 + j) * B + row] = v[j];
     }
-  }
-
-  // One 16-column chunk written straight from registers (row-major split
-  // and/or fp32, plus the mirror), or scattered.
-  __device__ __forceinline__ void chunk(const GemmOp& g, size_t B, size_t BB, int row, int col0, float* v,
-                                        const float* cj, bool mirror) {
-    apply(row, col0, v, cj);
-    if (scatter || of) check_finite(v);
-    if (scatter) {
-      scatter_chunk(g, row, col0, v);
-      return;
-    }
-    if (os) {
-      float w[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) w[j] = v[j] * ss;
-      store_split16(os, BB, row * B + col0, w, bad);
-    }
-    if (of) {
-      float4* d4 = reinterpret_cast<float4*>(of + row * B + col0);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    }
-    if (mirror) store_mirror(B, BB, row, col0, v);
   }
 
   // Warp-collective: the non-finite flag and the scattered sum of squares.

@@ -20,8 +20,9 @@
 // two buffers and there is no room to park a finished tile.  The accumulator
 // warps therefore write their own tile out.
 //
-// Shared memory: two 96 KB operand stages, 32 KB of epilogue staging, the
-// barriers (about 225 KB of the 227 KB a block may hold).
+// Shared memory: two 96 KB operand stages, 32 KB of epilogue staging (4 KB
+// per accumulator warp; stage 1 lends 12 KB more per warp during a tile's
+// epilogue), the barriers (about 225 KB of the 227 KB a block may hold).
 //
 // Roles (384 threads = three warpgroups, one CTA per SM, persistent over a
 // static round-robin list of the launch's tiles):
@@ -29,11 +30,11 @@
 //                      lanes 32*(w%4).. and 128 of the 256 columns, so each
 //                      thread sums 128 columns of one output row in
 //                      registers; at the end of a tile the same thread applies
-//                      the epilogue to its row segment.  Row-major outputs
-//                      leave through the warp's two 2 KB shared-memory
-//                      staging buffers, one TMA tensor store per 32 x 16
-//                      chunk (a store instruction whose 32 lanes each write
-//                      a different row would touch 32 lines).
+//                      the epilogue to its row segment, in four steps of 32
+//                      columns.  Each step leaves through a 4 KB shared-memory
+//                      buffer and one TMA tensor store (a store instruction
+//                      whose 32 lanes each write a different row would touch
+//                      32 lines); its Cin arrives in the same buffer by TMA.
 //   warp 8, one lane   TMA producer: A hi/lo (128 x 64) and B hi/lo
 //                      (256 x 64, or four 64 x 64 boxes when B is read
 //                      MN-major) of each 64-wide K slab into a 2-stage ring

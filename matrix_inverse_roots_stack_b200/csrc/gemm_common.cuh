@@ -281,6 +281,38 @@ __device__ __forceinline__ void stage_f32x32(uint8_t* buf, int lane, const float
   }
 }
 
+// The transpose of a step into a split staging buffer: lane l's value of
+// column j goes to row j, column l (v already times the split factor; the
+// non-finite check is the one stage_split32 made on the same values).  For
+// a fixed j the 32 lanes write one 64-byte row, so the stores do not
+// conflict.
+__device__ __forceinline__ void stage_split32_t(uint8_t* buf, int lane, const float (*v)[16]) {
+  const uint32_t col = static_cast<uint32_t>((lane & 7) * 2);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      __half2 hi, lo;
+      split_f16x2(v[c][j], v[c][j + 1], hi, lo);
+      const int r = 16 * c + j;  // rows r and r + 1 share the swizzle phase (r even)
+      const uint32_t o = static_cast<uint32_t>(r * 64 + (((lane >> 3) ^ ((r >> 1) & 3)) << 4)) + col;
+      *reinterpret_cast<__half*>(buf + o) = __low2half(hi);
+      *reinterpret_cast<__half*>(buf + o + 64) = __high2half(hi);
+      *reinterpret_cast<__half*>(buf + 2048 + o) = __low2half(lo);
+      *reinterpret_cast<__half*>(buf + 2048 + o + 64) = __high2half(lo);
+    }
+  }
+}
+
+// The transpose of a step into an fp32 staging buffer: lane l's value of
+// column j goes to row j, column l (one 128-byte row per j).
+__device__ __forceinline__ void stage_f32x32_t(uint8_t* buf, int lane, const float (*v)[16]) {
+  const uint32_t col = static_cast<uint32_t>((lane & 3) * 4);
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    *reinterpret_cast<float*>(buf + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) + col) = v[j >> 4][j & 15];
+}
+
 // Cin of chunk c (0, 1) of a step from a split staging buffer, joined to fp32
 __device__ __forceinline__ void read_cin_chunk(const uint8_t* buf, int lane, int c, float* cj) {
   SplitChunk r;
@@ -314,9 +346,6 @@ __device__ __forceinline__ void store_step(int lane, const CUtensorMap* map, con
   }
 }
 
-// kSingle: single-pass fp16 products (hi planes only, one MMA per K=16
-// step, a whole K slab per buffer; the fp16 coupled-Newton mode); otherwise
-// split-fp16 products with two K=16 steps per buffer.
 // A staged fp32 step (stage_f32x32) scattered into parameter layout: lane l
 // writes column col0 + l of rows row0.. (coalesced across the lanes), inside
 // the block's extent only, and adds its squares to sumsq.

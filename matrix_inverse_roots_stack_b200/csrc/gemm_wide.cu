@@ -498,6 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ep.scatter_chunk(g, row, col0 + 16, v[1]);
             continue;
           }
+          // a mirrored step also goes out transposed (rows col0.., columns
+          // row0..) through the same buffer, once the store before it has
+          // read the buffer
           if (ep.os) {
             float w[2][16];
 #pragma unroll
@@ -506,20 +509,28 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int j = 0; j < 16; ++j) w[h][j] = v[h][j] * ep.ss;
             stage_split32(buf, lane, w, ep.bad);
             store_step(lane, &om.split[op], buf, col0, row0, 2 * gemm_at(g.out_i, p));
+            if (mirror) {
+              if (lane == 0) bulk_wait_read<0>();
+              __syncwarp();
+              stage_split32_t(buf, lane, w);
+              store_step(lane, &om.split[op], buf, row0, col0, 2 * gemm_at(g.out_i, p));
+            }
           }
           if (ep.of) {
             ep.check_finite(v[0]);
             ep.check_finite(v[1]);
-            if (ep.os) {  // the split store must have read buf first
+            if (ep.os) {  // the split stores must have read buf first
               if (lane == 0) bulk_wait_read<0>();
               __syncwarp();
             }
             stage_f32x32(buf, lane, v);
             store_step(lane, &om.f32[op], buf, col0, row0, gemm_at(g.outf_i, p));
-          }
-          if (mirror) {
-            ep.store_mirror(B, BB, row, col0, v[0]);
-            ep.store_mirror(B, BB, row, col0 + 16, v[1]);
+            if (mirror) {
+              if (lane == 0) bulk_wait_read<0>();
+              __syncwarp();
+              stage_f32x32_t(buf, lane, v);
+              store_step(lane, &om.f32[op], buf, row0, col0, gemm_at(g.outf_i, p));
+            }
           }
         }
         if (!ok) {

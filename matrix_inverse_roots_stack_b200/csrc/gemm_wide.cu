@@ -153,6 +153,17 @@ __device__ __forceinline__ void decode_wide(const GemmArgs& args, int tpp, int n
   tj = row / 2 + r;
 }
 
+// This CTA's tile in round k of the launch's static schedule.  Round k
+// covers tiles k*G .. k*G + G - 1 (G CTAs), and a CTA's place in the round
+// moves by one each round, so tiles that recur at fixed places in every
+// problem's tile list (the half-width tiles of symmetric launches) are
+// spread over all CTAs instead of falling to the same few.  A result at or
+// past the launch's total is a place in the last round with no tile.
+__device__ __forceinline__ long long round_tile(long long k) {
+  const long long g = gridDim.x;
+  return k * g + (static_cast<long long>(blockIdx.x) + k) % g;
+}
+
 // L2 prefetch of one row segment [cbase, cbase + kCols) of problem p's Cin
 // (split hi and lo planes, or fp32): 128-byte lines, no registers held.
 __device__ __forceinline__ void prefetch_cin_l2(const GemmOp& g, int p, size_t B, size_t BB, int row, int cbase) {
@@ -229,8 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sc = 0, s = 0, epar = 1;  // loads issued, stage, parity of the stage's next release
       uint32_t fpar = 0;                 // parity of the next stg_free phase
       bool stop = args.skip_loads != 0;
-      for (long long t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-        const bool after_epilogue = t != blockIdx.x;  // stage 1 holds the previous tile's epilogue staging
+      bool first = true;
+      for (long long k = 0; k * gridDim.x < total && !stop; ++k) {
+        const long long t = round_tile(k);
+        if (t >= total) continue;
+        const bool after_epilogue = !first;  // stage 1 holds the previous tile's epilogue staging
+        first = false;
         int op, p, ti, tj;
         decode_wide(args, tpp, ntn, t, op, p, ti, tj);
         const GemmOp& g = args.op[op];
@@ -285,12 +300,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t s = 0, fpar = 0;                   // stage, parity of its next fill
       uint32_t hb = 0, hpar = (1u << kRing) - 1u;  // ring buffer, parity bits of the next release per buffer
       bool ok = true;
-      for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (long long k = 0; k * gridDim.x < total && ok; ++k) {
+        const long long t = round_tile(k);
+        if (t >= total) continue;
         int op, p, ti, tj;
         decode_wide(args, tpp, ntn, t, op, p, ti, tj);
         const bool bmn = args.op[op].b_mn != 0;
-        const uint32_t idesc = f16_idesc(kM, kN) | (bmn ? (1u << 16) : 0u);
-        const uint64_t bd0 = (bmn ? md0 : kd0) + 2 * kAD;
+        // a symmetric launch keeps nothing of a tile's left half below the
+        // diagonal (the first tile of an odd tile row): its MMAs compute the
+        // right half only (N=128, B rows 128.., tensor-memory columns 128..)
+        const bool half = args.sym && 2 * tj < ti;
+        const uint32_t idesc = f16_idesc(kM, half ? kN / 2 : kN) | (bmn ? (1u << 16) : 0u);
+        const uint64_t bd0 = (bmn ? md0 : kd0) + 2 * kAD + (half ? (kBBytes / 2) >> 4 : 0);
+        const uint32_t dcol = half ? kN / 2 : 0;
         const uint32_t bstep = bmn ? (2048u >> 4) : (32u >> 4);
         for (int kb = 0; kb < nk; ++kb) {
           ok = mbar_wait(&bars->full[s], fpar, abort_flag);
@@ -304,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             hpar ^= 1u << hb;
             if (!ok) break;
             tc_fence_after();
-            const uint32_t d = tbase + hb * kN;
+            const uint32_t d = tbase + hb * kN + dcol;
             const int k0 = f * kFillSteps;
             if (kSingle) {  // hi*hi of the slab's four steps into a fresh buffer
 #pragma unroll
@@ -354,7 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool cin0_pending = false;  // a Cin load of this warp has not been waited for (own buffer,
     bool cin_pending = false;   // stage 1)
     bool ok = true;
-    for (long long t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (long long k = 0; k * gridDim.x < total && ok; ++k) {
+      const long long t = round_tile(k);
+      if (t >= total) continue;
       float S[kCols];
 #pragma unroll
       for (int j = 0; j < kCols; ++j) S[j] = 0.0f;
@@ -397,6 +421,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         hpar ^= 1u << hb;
         tc_fence_after();
+        if (!write) {  // nothing of this half is kept (and the MMA may not have written it)
+          if (sg + 1 < nfill) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[hb]);
+            hb ^= 1u;
+          }
+          continue;
+        }
         const uint32_t src = tbase + lane_off + hb * kN;
         if (sg + 1 < nfill) {
 #pragma unroll

@@ -44,11 +44,11 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 # DRAM bytes (read + write) per executed tensor-core flop of the GEMM, by
 # (kernel, block size, solver): from an ncu capture of every launch of three
 # steps of the mixed-shape B=1024 workload (24 factors of 1024, Newton-DB
-# 14 + 14): 59.68 GB over 3.69e13 executed flops.  Each launch reads and writes
+# 14 + 14): 59.82 GB over 3.69e13 executed flops.  Each launch reads and writes
 # its problems' split matrices about once, so a launch's traffic grows in
 # proportion to the problems, and executed flops, it covers; the roofline's
 # per-launch traffic scales this ratio by those flops.
-GEMM_DRAM_BYTES_PER_FLOP = {("gemm_wide_kernel", 1024, "ndb"): 1.616e-3}
+GEMM_DRAM_BYTES_PER_FLOP = {("gemm_wide_kernel", 1024, "ndb"): 1.622e-3}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

@@ -674,9 +674,11 @@ cudaError_t launch_gemm_wide(const CUtensorMap* maps, const GemmArgs& a, long lo
   const long long sms = gemm_sm_count();
   const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
   // executed tensor-core flops: each 128 x 256 tile is one 2*128*256*B
-  // product, done as three fp16 products (one in single-pass mode)
-  const double flops =
-      (a.single_pass ? 1.0 : 3.0) * 2.0 * kM * kN * static_cast<double>(a.B) * static_cast<double>(total);
+  // product, done as three fp16 products (one in single-pass mode); in a
+  // symmetric launch the first tile of each odd tile row (B/256 a problem)
+  // runs at half width
+  const double full_tiles = static_cast<double>(total) - (a.sym ? 0.5 * (a.B / kN) * static_cast<double>(nprob) : 0.0);
+  const double flops = (a.single_pass ? 1.0 : 3.0) * 2.0 * kM * kN * static_cast<double>(a.B) * full_tiles;
   for (int o = 0; o < a.nops; ++o)  // a scattering op reads no Cin on 128 x 256 tiles
     if (a.op[o].nprob > 0 && a.op[o].blocks && (a.op[o].cin_split || a.op[o].cin_f32)) return cudaErrorInvalidValue;
   OutMaps om;

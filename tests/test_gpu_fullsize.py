@@ -26,7 +26,7 @@ import pytest
 
 from matrix_inverse_roots_stack_b200 import workloads
 from oracle import step as ostep
-from tests.gpu_util import rel, cuda_or_skip
+from tests.gpu_util import assert_mirrored_blocks, rel, cuda_or_skip
 
 pytestmark = pytest.mark.gpu
 
@@ -80,6 +80,7 @@ def run_and_check(torch, shapes, grads, B, solver="ndb", iters=14, degree=16, n_
     opt.step()
     rc, flags = opt.status()
     assert rc == 0, bd.strerror(rc)
+    assert_mirrored_blocks(torch, opt.factors)
     lam = opt.lam.cpu().numpy().astype(np.float64)
     table = opt.block_table()
     hp = ostep.HParams(block_size=B, solver=solver, ndb_iters1=iters, ndb_iters2=iters, cheb_degree=degree,

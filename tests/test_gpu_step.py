@@ -11,7 +11,7 @@ import pytest
 
 from matrix_inverse_roots_stack_b200 import workloads
 from oracle import step as ostep, roots
-from tests.gpu_util import rel, cuda_or_skip
+from tests.gpu_util import assert_mirrored_blocks, rel, cuda_or_skip
 
 pytestmark = pytest.mark.gpu
 
@@ -180,6 +180,8 @@ def test_two_steps_block_256(torch):
     hp = ostep.HParams(block_size=256, ndb_iters1=14, ndb_iters2=14, eps=1e-5)
     gpu = run_gpu(torch, th, grads, hp, steps=2)
     compare(gpu, th, grads, hp, steps=2)
+    for F in gpu["factors"]:  # the factor update is a symmetric launch
+        assert_mirrored_blocks(torch, torch.from_numpy(F))
 
 
 def test_root_every_reuses_roots(torch):

@@ -70,12 +70,13 @@ def sample_blocks(table, n_sample):
 
 
 def run_and_check(torch, shapes, grads, B, solver="ndb", iters=14, degree=16, n_sample=MIN_SAMPLE, eps=1e-6,
-                  require_regime=False, flat=True):
+                  require_regime=False, flat=True, cn_iters=16):
     from matrix_inverse_roots_stack_b200 import binding as bd
     dev = grads[0].device
     params = [torch.zeros_like(g) for g in grads]
-    hpb = bd.make_hparams(block_size=B, solver=bd.SOLVER_NEWTON_DB if solver == "ndb" else bd.SOLVER_CHEBYSHEV,
-                          ndb_iters1=iters, ndb_iters2=iters, cheb_degree=degree, eps=eps)
+    code = {"ndb": bd.SOLVER_NEWTON_DB, "cheb": bd.SOLVER_CHEBYSHEV, "cn": bd.SOLVER_COUPLED_NEWTON}[solver]
+    hpb = bd.make_hparams(block_size=B, solver=code, ndb_iters1=iters, ndb_iters2=iters, cheb_degree=degree,
+                          eps=eps, cn_iters=cn_iters)
     opt = bd.Shampoo(params, grads, hp=hpb, v0=torch.from_numpy(workloads.pi_start_vectors(B, 32, seed=0)).to(dev))
     opt.step()
     rc, flags = opt.status()
@@ -84,7 +85,7 @@ def run_and_check(torch, shapes, grads, B, solver="ndb", iters=14, degree=16, n_
     lam = opt.lam.cpu().numpy().astype(np.float64)
     table = opt.block_table()
     hp = ostep.HParams(block_size=B, solver=solver, ndb_iters1=iters, ndb_iters2=iters, cheb_degree=degree,
-                       beta=f32(0.95), eps=f32(eps), init_scale=f32(1e-6), beta1=f32(0.9), beta2=f32(0.999),
+                       cn_iters=cn_iters, beta=f32(0.95), eps=f32(eps), init_scale=f32(1e-6), beta1=f32(0.9), beta2=f32(0.999),
                        adam_eps=f32(1e-8), lr=f32(1e-3), cheb_delta=f32(1e-3))
     rows = []
     for k in sample_blocks(table, n_sample):
@@ -145,6 +146,13 @@ def test_llama_1b_b1024_chebyshev_d60(torch):
     shapes = workloads.llama_1b_shapes()
     grads = workloads.torch_gaussian_gradients(shapes, "cuda", std=0.1, seed=0, row_lognormal_sigma=1.0)
     run_and_check(torch, shapes, grads, 1024, solver="cheb", degree=60)
+
+
+def test_llama_1b_b1024_coupled_newton(torch):
+    # split-fp16 coupled Newton, 16 iterations, on upper-triangle tiles
+    shapes = workloads.llama_1b_shapes()
+    grads = workloads.torch_gaussian_gradients(shapes, "cuda", std=0.1, seed=0, row_lognormal_sigma=1.0)
+    run_and_check(torch, shapes, grads, 1024, solver="cn")
 
 
 @pytest.mark.parametrize("B", [256, 1024, 2048])

@@ -142,10 +142,11 @@ def test_mixed_shapes_chebyshev(torch, B, degree):
     run_and_check(torch, shapes, grads, B, solver="cheb", degree=degree, flat=False)
 
 
-def test_llama_1b_b1024_chebyshev_d60(torch):
+@pytest.mark.parametrize("degree", [16, 60])
+def test_llama_1b_b1024_chebyshev(torch, degree):
     shapes = workloads.llama_1b_shapes()
     grads = workloads.torch_gaussian_gradients(shapes, "cuda", std=0.1, seed=0, row_lognormal_sigma=1.0)
-    run_and_check(torch, shapes, grads, 1024, solver="cheb", degree=60)
+    run_and_check(torch, shapes, grads, 1024, solver="cheb", degree=degree)
 
 
 def test_llama_1b_b1024_coupled_newton(torch):

@@ -547,7 +547,8 @@ def main():
     # ---------------- roofline of the dominant kernel (a split-fp16 GEMM)
     peaks, peak_kind = load_peaks()
     tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    kernels = {"gemm_wide_kernel": prof["gemm_wide"], "gemm_split_kernel": prof["gemm"]}
+    kernels = {"gemm_wide_kernel": prof["gemm_wide"], "gemm_split_kernel": prof["gemm"],
+               "ndb_fused_kernel": prof["ndb_fused"]}
 
     def kernel_line(ms_, n_, fl_):
         avg = ms_ / max(n_, 1)
@@ -602,7 +603,7 @@ def main():
                         "frac_of_tf32_peak_unpadded": round(unpadded / root_s / 1e12 / tf32_peak, 4),
                         "peak_kind": f"{peak_kind}: bf16 sustained x 0.5 (nominal TF32/BF16 ratio)"}
     stages = {k: round(v[0] / prof_steps, 3) for k, v in prof.items()
-              if isinstance(v, tuple) and k not in ("gemm", "gemm_wide")}
+              if isinstance(v, tuple) and k not in ("gemm", "gemm_wide", "ndb_fused")}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:

@@ -283,17 +283,19 @@ SHAMPOO_API const char* shampoo_strerror(int code);
 SHAMPOO_API int shampoo_profile_enable(int enable);
 /* Forget everything recorded so far. */
 SHAMPOO_API int shampoo_profile_reset(void);
-/* Synchronise the recorded events and fill out[0 .. 23]:
+/* Synchronise the recorded events and fill out[0 .. 26]:
  * out[3s], out[3s+1], out[3s+2] = milliseconds, count and flops of stage s,
  * for s = 0 launches of the tensor-core GEMM with 128 x 128 tiles (executed
  * tensor-core flops: 3 * 2*128*128*B per computed tile, or 1 * ... for
  * single-pass fp16 launches), 1 gather + factor EMA, 2 power iteration,
  * 3 root solver, 4 preconditioner products, 5 Adam graft + update, 6 launches
- * of the tensor-core GEMM with 128 x 256 tiles (3 * 2*128*256*B per tile);
- * out[21] = kernel launches since the last reset; out[22] = records dropped;
- * out[23] = registers a thread of the 128 x 256 kernel was compiled with (it
+ * of the tensor-core GEMM with 128 x 256 tiles (3 * 2*128*256*B per tile), 7
+ * launches of the Newton-DB kernel on resident factors of 128 (9 * 2*128^3
+ * per iteration and factor);
+ * out[24] = kernel launches since the last reset; out[25] = records dropped;
+ * out[26] = registers a thread of the 128 x 256 kernel was compiled with (it
  * is used only when that is 168, the count its register split assumes).
- * n >= 24. */
+ * n >= 27. */
 SHAMPOO_API int shampoo_profile_read(double* out, int n);
 
 /* Test hook for the failure path (not part of the method): arms a one-shot

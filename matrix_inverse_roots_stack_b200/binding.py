@@ -219,7 +219,8 @@ def read_static_status(stream=None):
     return rc, flags.value
 
 
-PROFILE_STAGES = ("gemm", "accumulate", "power_iteration", "solver", "precondition", "adam_update", "gemm_wide")
+PROFILE_STAGES = ("gemm", "accumulate", "power_iteration", "solver", "precondition", "adam_update", "gemm_wide",
+                  "ndb_fused")
 
 
 def profile_enable(on=True):

@@ -175,7 +175,12 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
     return SHAMPOO_OK;
   };
   auto iterate = [&](int T, bool final_stage) -> int {
-    for (int it = 1; it < T; ++it) {
+    int it = 1;
+    if (B == 128 && T > 2) {  // the middle iterations on factors held in shared memory, in place
+      DASH_TRY(dash::launch_ndb_fused(Yb[yc], Zb[zc], n, B, -0.5f * kZScale, T - 2, status, st));
+      it = T - 1;
+    }
+    for (; it < T; ++it) {
       {  // D = (I - zs Zhat Y)/2   (A = Zhat, B = Y)
         GemmArgs g = gemm_args(B, 0, status);
         dash::GemmOp& o = g.op[0];

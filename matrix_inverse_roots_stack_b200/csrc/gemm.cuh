@@ -89,6 +89,14 @@ struct OpBuffers {
 // launch / encode error.
 cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaStream_t stream);
 
+// Newton-DB iterations on a stack of n factors of 128 held in shared memory
+// (one CTA per factor): `iters` times D = alpha_d Zhat Y + I/2, Y <- Y + Y D,
+// Zhat <- Zhat + D Zhat, in place on the split stacks Y and Zhat (layout as
+// OpBuffers); the products' arithmetic is that of launch_gemm_split.
+// Returns cudaErrorNotSupported unless B == 128.
+cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, int n, int B, float alpha_d, int iters, unsigned* status,
+                             cudaStream_t stream);
+
 // Arm a one-shot test fault: the next GEMM launch withholds its operand loads,
 // so its waits run into their time limit and it reports a timeout.
 void arm_load_fault();

@@ -24,13 +24,14 @@ __device__ __forceinline__ void gemm_fail_timeout(volatile int* abort_flag, unsi
   if (status) atomicOr(status, kStatusTimeout);
 }
 
-// Descriptor of an MN-major operand tile: 64 K-rows of 128 bytes per
-// 64-column box, boxes 8 KB apart (leading byte offset), 8-row swizzle atoms
-// of 1024 bytes (stride byte offset), 128-byte swizzle.
-__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
+// Descriptor of an MN-major operand tile: K-rows of 128 bytes (64 columns)
+// per block, blocks block_bytes apart (leading byte offset; 8 KB for blocks
+// of 64 K-rows), 8-row swizzle atoms of 1024 bytes (stride byte offset),
+// 128-byte swizzle.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t block_bytes = 8192u) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(8192u >> 4) << 16;
+  d |= static_cast<uint64_t>(block_bytes >> 4) << 16;
   d |= static_cast<uint64_t>(1024u >> 4) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;

@@ -18,7 +18,8 @@ enum ProfStage {
   kProfPrecond = 4,      // U = X_L G X_R
   kProfAdam = 5,         // Adam moments, graft and update
   kProfGemmWide = 6,     // launches of the split-fp16 GEMM with 128 x 256 tiles (gemm_wide.cu)
-  kProfStages = 7
+  kProfNdbFused = 7,     // launches of the Newton-DB kernel on resident 128 x 128 factors (ndb_fused.cu)
+  kProfStages = 8
 };
 
 bool prof_on();

@@ -174,13 +174,8 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
     yc ^= 1;
     return SHAMPOO_OK;
   };
-  auto iterate = [&](int T, bool final_stage) -> int {
-    int it = 1;
-    if (B == 128 && T > 2) {  // the middle iterations on factors held in shared memory, in place
-      DASH_TRY(dash::launch_ndb_fused(Yb[yc], Zb[zc], n, B, -0.5f * kZScale, T - 2, status, st));
-      it = T - 1;
-    }
-    for (; it < T; ++it) {
+  auto iterate = [&](int it0, int T, bool final_stage) -> int {
+    for (int it = it0; it < T; ++it) {
       {  // D = (I - zs Zhat Y)/2   (A = Zhat, B = Y)
         GemmArgs g = gemm_args(B, 0, status);
         dash::GemmOp& o = g.op[0];
@@ -219,10 +214,20 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
     return SHAMPOO_OK;
   };
 
-  int rc = first_y();
-  if (rc) return rc;
-  rc = iterate(it1, false);
-  if (rc) return rc;
+  // at B = 128 a factor's iterates fit in one SM's shared memory: a stage's
+  // iterations up to its last run there, in place on Y and Zhat
+  const bool resident = B == 128;
+  const float alpha_d = -0.5f * kZScale;
+  int rc = SHAMPOO_OK;
+  if (resident) {
+    DASH_TRY(dash::launch_ndb_fused(Yb[yc], Zb[zc], D, n, B, alpha_d, 1, it1 >= 2 ? it1 - 2 : 0, it1 >= 2 ? 1 : 0,
+                                    status, st));
+  } else {
+    rc = first_y();
+    if (rc) return rc;
+    rc = iterate(1, it1, false);
+    if (rc) return rc;
+  }
   // stage 2 on Y: D0 = (I - Y)/2, Zhat1 = (I + D0)/zs, Y1 = Y + Y D0
   dash::launch_ndb_stage2_init(Yb[yc], n, B, kZScale, D, Zb[zc], st);
   DASH_LAUNCHED();
@@ -231,9 +236,13 @@ int run_ndb_chunk(const float* F, int n, int B, float eps, const int* fsize, con
     DASH_LAUNCHED();
     return SHAMPOO_OK;
   }
+  if (resident) {
+    DASH_TRY(dash::launch_ndb_fused(Yb[yc], Zb[zc], D, n, B, alpha_d, 1, it2 - 2, 0, status, st));
+    return iterate(it2 - 1, it2, true);
+  }
   rc = first_y();
   if (rc) return rc;
-  return iterate(it2, true);
+  return iterate(1, it2, true);
 }
 
 // Chebyshev / Clenshaw on one chunk ("Building blocks", Chebyshev; the

@@ -90,12 +90,15 @@ struct OpBuffers {
 cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaStream_t stream);
 
 // Newton-DB iterations on a stack of n factors of 128 held in shared memory
-// (one CTA per factor): `iters` times D = alpha_d Zhat Y + I/2, Y <- Y + Y D,
-// Zhat <- Zhat + D Zhat, in place on the split stacks Y and Zhat (layout as
-// OpBuffers); the products' arithmetic is that of launch_gemm_split.
-// Returns cudaErrorNotSupported unless B == 128.
-cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, int n, int B, float alpha_d, int iters, unsigned* status,
-                             cudaStream_t stream);
+// (one CTA per factor), in place on the split stacks Y and Zhat (layout as
+// OpBuffers), in this order: if first, Y <- Y + Y D with D read from the
+// split stack D; `iters` times D = alpha_d Zhat Y + I/2, Y <- Y + Y D,
+// Zhat <- Zhat + D Zhat; if last_y, once more D = alpha_d Zhat Y + I/2,
+// Y <- Y + Y D (Zhat is then left as it was).  The products' arithmetic is
+// that of launch_gemm_split.  Returns cudaErrorNotSupported unless B == 128
+// and first, last_y are 0 or 1.
+cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, const __half* D, int n, int B, float alpha_d, int first,
+                             int iters, int last_y, unsigned* status, cudaStream_t stream);
 
 // Arm a one-shot test fault: the next GEMM launch withholds its operand loads,
 // so its waits run into their time limit and it reports a timeout.

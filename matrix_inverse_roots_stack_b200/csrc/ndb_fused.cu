@@ -4,10 +4,12 @@
 // updates Y <- Y + Y D, Z <- Z + D Z (E = I + D applied in correction
 // form, products in the page's order; Z is kept as Zhat = Z / zs).  At
 // B = 128 a factor's Y, Zhat and D, as split fp16 (hi and lo planes), take
-// 3 x 64 KB: one CTA keeps them in shared memory and runs a stage's middle
-// iterations on them with no trip through HBM and no launch per product.
-// The first and last iterations of a stage, which have their own forms, stay
-// on the batched GEMM.
+// 3 x 64 KB: one CTA keeps them in shared memory and runs a stage's
+// iterations on them with no trip through HBM and no launch per product:
+// the first (Y + Y D0, D0 from the stage's prologue), the full middle ones,
+// and a last one that updates Y only.  The final iteration of the second
+// stage, whose output is the root in fp32 and split form, stays on the
+// batched GEMM.
 //
 // Arithmetic: the same as the 128 x 128 GEMM, step for step.  Every K=16
 // step of a product is three tcgen05.mma kind::f16 (hi*lo, + lo*hi, then
@@ -25,17 +27,17 @@
 // next product's operand as it stands.
 //
 // Roles (320 threads, one CTA per SM, persistent over the factors):
-//   warp 0, one lane   loads a factor's Y and Zhat by TMA and stores them
-//                      back when its iterations are done;
+//   warp 0, one lane   loads a factor's Y and Zhat (and D0) by TMA and
+//                      stores them back when its iterations are done;
 //   warp 1, one lane   MMA issuer (warp 1 owns the tensor memory);
 //   warps 2-9          accumulators: warp w reads tensor-memory lanes
 //                      32*(w%4).. and 64 of the 128 columns, sums them per
 //                      row in registers, and writes D, Y and Zhat back into
 //                      shared memory (then a proxy fence, so that the tensor
 //                      core reads what they wrote).
-// Per iteration the MMA issues 24 steps (D = Zhat Y, then Y D, then D Zhat)
-// through a ring of four buffers; it waits for D before the second product
-// and for Y and Zhat before the next iteration's first.
+// Per full iteration the MMA issues 24 steps (D = Zhat Y, then Y D, then
+// D Zhat) through a ring of four buffers; it waits for D before the second
+// product and for Y and Zhat before the next iteration's first.
 #include "gemm.cuh"
 #include "gemm_common.cuh"
 #include "launch_util.cuh"
@@ -71,6 +73,24 @@ struct Bars {
   int abort;
 };
 constexpr int kBarsOff = 3 * kMatBytes;
+
+// Steps of one launch, the same for every factor: groups run in order, each
+// ending with Y (and Zhat) back in shared memory.
+//   first   Y <- Y + Y D, with D loaded from HBM beside Y and Zhat (a
+//           stage's first iteration, whose D comes from its prologue);
+//   iters   full iterations: D = alpha_d Zhat Y + I/2, Y <- Y + Y D,
+//           Zhat <- Zhat + D Zhat;
+//   last_y  one more iteration that updates Y only (the last of a stage
+//           whose Zhat is not used afterwards).
+struct FusedPlan {
+  int first, iters, last_y;
+};
+enum GroupKind { kFirstY = 0, kFull = 1, kLastY = 2 };
+__host__ __device__ __forceinline__ int plan_groups(const FusedPlan& pl) { return pl.first + pl.iters + pl.last_y; }
+__device__ __forceinline__ int group_kind(const FusedPlan& pl, int gi) {
+  if (pl.first && gi == 0) return kFirstY;
+  return pl.last_y && gi == plan_groups(pl) - 1 ? kLastY : kFull;
+}
 constexpr int kSmemBytes = kBarsOff + static_cast<int>(sizeof(Bars)) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory exceeds the per-block limit");
 static_assert(kRing * 128 <= static_cast<int>(kTmemCols), "ring exceeds tensor memory");
@@ -146,8 +166,9 @@ __device__ __forceinline__ void write_row(uint8_t* buf, int cb, int r, const flo
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    ndb_fused_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmZ, const int n,
-                     const float alpha_d, const int iters, unsigned* status) {
+    ndb_fused_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmZ,
+                     const __grid_constant__ CUtensorMap tmD, const int n, const float alpha_d, const FusedPlan plan,
+                     unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -169,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmY);
     tma_prefetch_desc(&tmZ);
+    tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_slot, kTmemCols);
@@ -178,6 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = bars->tmem_slot;
+  const int groups = plan_groups(plan);
+  // Zhat changes only in full iterations, and is stored back when the last
+  // group is one
+  const bool store_z = group_kind(plan, groups - 1) == kFull;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- loads and stores
@@ -193,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cb = 0; cb < 2; ++cb) {
             const uint32_t o = pl * kPlaneBytes + cb * kColBlk;
             tma_store_3d(&tmY, smem + kYOff + o, 64 * cb, 0, 2 * p + pl);
-            tma_store_3d(&tmZ, smem + kZOff + o, 64 * cb, 0, 2 * p + pl);
+            if (store_z) tma_store_3d(&tmZ, smem + kZOff + o, 64 * cb, 0, 2 * p + pl);
           }
         bulk_commit();
       };
@@ -205,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           store(prev);
           bulk_wait_read<0>();
         }
-        mbar_arrive_expect_tx(&bars->ld_full, 2 * kMatBytes);
+        mbar_arrive_expect_tx(&bars->ld_full, (plan.first ? 3 : 2) * kMatBytes);
 #pragma unroll
         for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
@@ -213,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t o = pl * kPlaneBytes + cb * kColBlk;
             tma_load_3d(smem + kYOff + o, &tmY, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
             tma_load_3d(smem + kZOff + o, &tmZ, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
+            if (plan.first) tma_load_3d(smem + kDOff + o, &tmD, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
           }
         ++loads;
         prev = t;
@@ -254,12 +281,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         lpar ^= 1u;
         if (!ok) break;
         tc_fence_after();
-        for (int it = 0; it < iters && ok; ++it) {
-          if (it > 0) {  // Y and Zhat of the previous iteration are back
+        for (int gi = 0; gi < groups && ok; ++gi) {
+          const int kind = group_kind(plan, gi);
+          if (gi > 0) {  // Y and Zhat of the previous group are back
             ok = mbar_wait(&bars->yz_ready, ypar, abort_flag);
             ypar ^= 1u;
             if (!ok) break;
             tc_fence_after();
+          }
+          if (kind == kFirstY) {
+            ok = product(kYOff, kDOff);  // Y D0
+            continue;
           }
           ok = product(kZOff, kYOff);  // Zhat Y
           if (!ok) break;
@@ -267,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           dpar ^= 1u;
           if (!ok) break;
           tc_fence_after();
-          ok = product(kYOff, kDOff) && product(kDOff, kZOff);  // Y D, then D Zhat
+          ok = product(kYOff, kDOff);  // Y D
+          if (ok && kind == kFull) ok = product(kDOff, kZOff);  // D Zhat
         }
       }
       if (!ok) gemm_fail_timeout(abort_flag, status);
@@ -317,25 +350,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the factor's Y and Zhat (the first Cin) come from the TMA load
       ok = __all_sync(0xffffffffu, mbar_wait_sleep(&bars->ld_full, lpar, abort_flag));
       lpar ^= 1u;
-      for (int it = 0; it < iters && ok; ++it) {
+      for (int gi = 0; gi < groups && ok; ++gi) {
+        const int kind = group_kind(plan, gi);
         float S[kCols];
-        ok = flush(S);  // Zhat Y
-        if (!ok) break;
-        write_row(smem + kDOff, cgrp, r, S, alpha_d, false, 0.5f, bad);  // D = alpha_d Zhat Y + I/2
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->d_ready);
+        if (kind != kFirstY) {
+          ok = flush(S);  // Zhat Y
+          if (!ok) break;
+          write_row(smem + kDOff, cgrp, r, S, alpha_d, false, 0.5f, bad);  // D = alpha_d Zhat Y + I/2
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->d_ready);
+        }
         // Y D's MMAs are done once its last step is here, so Y may be
         // rewritten (D Zhat, still running, does not read Y)
         ok = flush(S);
         if (!ok) break;
         write_row(smem + kYOff, cgrp, r, S, 1.0f, true, 0.0f, bad);  // Y + Y D
-        ok = flush(S);  // D Zhat
-        if (!ok) break;
-        write_row(smem + kZOff, cgrp, r, S, 1.0f, true, 0.0f, bad);  // Zhat + D Zhat
+        if (kind == kFull) {
+          ok = flush(S);  // D Zhat
+          if (!ok) break;
+          write_row(smem + kZOff, cgrp, r, S, 1.0f, true, 0.0f, bad);  // Zhat + D Zhat
+        }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(it + 1 < iters ? &bars->yz_ready : &bars->yz_final);
+        if (lane == 0) mbar_arrive(gi + 1 < groups ? &bars->yz_ready : &bars->yz_final);
       }
     }
     if (!ok && lane == 0) gemm_fail_timeout(abort_flag, status);
@@ -352,24 +390,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, int n, int B, float alpha_d, int iters, unsigned* status,
-                             cudaStream_t stream) {
-  if (B != kN) return cudaErrorNotSupported;
-  if (n <= 0 || iters <= 0) return cudaSuccess;
-  CUtensorMap my, mz;
+cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, const __half* D, int n, int B, float alpha_d, int first,
+                             int iters, int last_y, unsigned* status, cudaStream_t stream) {
+  if (B != kN || iters < 0 || (first != 0 && first != 1) || (last_y != 0 && last_y != 1))
+    return cudaErrorNotSupported;
+  const FusedPlan plan{first, iters, last_y};
+  if (n <= 0 || plan_groups(plan) == 0) return cudaSuccess;
+  CUtensorMap my, mz, md;
   cudaError_t e = encode_split_stack_map(&my, Y, kN, n, kN);
   if (e != cudaSuccess) return e;
   e = encode_split_stack_map(&mz, Zhat, kN, n, kN);
+  if (e != cudaSuccess) return e;
+  e = encode_split_stack_map(&md, D, kN, n, kN);
   if (e != cudaSuccess) return e;
   static std::atomic<unsigned long long> attr_set;
   e = smem_limit_once(ndb_fused_kernel, kSmemBytes, attr_set);
   if (e != cudaSuccess) return e;
   const int sms = gemm_sm_count();
   const unsigned grid = static_cast<unsigned>(n < sms ? n : sms);
-  // executed tensor-core flops: three products of 2*128^3, three fp16 MMAs each
-  const double flops = 9.0 * 2.0 * kN * kN * static_cast<double>(kN) * iters * static_cast<double>(n);
+  // executed tensor-core flops: products of 2*128^3 (one for first, three
+  // per full iteration, two for last_y), three fp16 MMAs each
+  const double products = first + 3.0 * iters + 2.0 * last_y;
+  const double flops = 3.0 * 2.0 * kN * kN * static_cast<double>(kN) * products * static_cast<double>(n);
   const int slot = prof_begin(kProfNdbFused, stream, flops);
-  ndb_fused_kernel<<<grid, kThreads, kSmemBytes, stream>>>(my, mz, n, alpha_d, iters, status);
+  ndb_fused_kernel<<<grid, kThreads, kSmemBytes, stream>>>(my, mz, md, n, alpha_d, plan, status);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

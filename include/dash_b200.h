@@ -299,8 +299,8 @@ SHAMPOO_API int shampoo_profile_reset(void);
 SHAMPOO_API int shampoo_profile_read(double* out, int n);
 
 /* Test hook for the failure path (not part of the method): arms a one-shot
- * fault so that the next tensor-core GEMM launch withholds its operand
- * loads.  Its bounded waits then expire (about 2 s), the kernel sets
+ * fault so that the next launch of a tensor-core product kernel (the GEMM,
+ * or Newton-DB on resident factors of 128) withholds its operand loads.  Its bounded waits then expire (about 2 s), the kernel sets
  * SHAMPOO_STATUS_TIMEOUT in the workspace status word, releases its tensor
  * memory and returns; the context stays usable.  The results of that call
  * are undefined. */

@@ -439,7 +439,7 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
   if (args.B % kTile != 0 || args.B <= 0) return cudaErrorInvalidValue;
   GemmArgs a = args;
   if (a.nops == 1) a.op[1] = a.op[0], a.op[1].nprob = 0;
-  if (g_load_fault.exchange(0) != 0) a.skip_loads = 1;
+  if (take_load_fault()) a.skip_loads = 1;
   const bool wide = gemm_wide_supported(a);
   CUtensorMap maps[4];
   for (int o = 0; o < 2; ++o) {
@@ -475,5 +475,7 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
 }
 
 void arm_load_fault() { g_load_fault.store(1); }
+
+bool take_load_fault() { return g_load_fault.exchange(0) != 0; }
 
 }  // namespace dash

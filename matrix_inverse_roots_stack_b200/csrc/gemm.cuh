@@ -100,8 +100,11 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
 cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, const __half* D, int n, int B, float alpha_d, int first,
                              int iters, int last_y, unsigned* status, cudaStream_t stream);
 
-// Arm a one-shot test fault: the next GEMM launch withholds its operand loads,
+// Arm a one-shot test fault: the next launch of a tensor-core product kernel
+// (the GEMM, or Newton-DB on resident factors) withholds its operand loads,
 // so its waits run into their time limit and it reports a timeout.
 void arm_load_fault();
+// Consume the armed fault: true once after arm_load_fault.
+bool take_load_fault();
 
 }  // namespace dash

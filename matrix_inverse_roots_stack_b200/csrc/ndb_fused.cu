@@ -168,7 +168,7 @@ __device__ __forceinline__ void write_row(uint8_t* buf, int cb, int r, const flo
 __global__ void __launch_bounds__(kThreads, 1)
     ndb_fused_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmZ,
                      const __grid_constant__ CUtensorMap tmD, const int n, const float alpha_d, const FusedPlan plan,
-                     unsigned* status) {
+                     const int skip_loads, unsigned* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -231,17 +231,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           store(prev);
           bulk_wait_read<0>();
         }
-        mbar_arrive_expect_tx(&bars->ld_full, (plan.first ? 3 : 2) * kMatBytes);
+        if (!skip_loads) {  // (test hook: with skip_loads the operands never arrive)
+          mbar_arrive_expect_tx(&bars->ld_full, (plan.first ? 3 : 2) * kMatBytes);
 #pragma unroll
-        for (int pl = 0; pl < 2; ++pl)
+          for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-          for (int cb = 0; cb < 2; ++cb) {
-            const uint32_t o = pl * kPlaneBytes + cb * kColBlk;
-            tma_load_3d(smem + kYOff + o, &tmY, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
-            tma_load_3d(smem + kZOff + o, &tmZ, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
-            if (plan.first) tma_load_3d(smem + kDOff + o, &tmD, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
-          }
-        ++loads;
+            for (int cb = 0; cb < 2; ++cb) {
+              const uint32_t o = pl * kPlaneBytes + cb * kColBlk;
+              tma_load_3d(smem + kYOff + o, &tmY, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
+              tma_load_3d(smem + kZOff + o, &tmZ, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
+              if (plan.first) tma_load_3d(smem + kDOff + o, &tmD, &bars->ld_full, 64 * cb, 0, 2 * t + pl);
+            }
+          ++loads;
+        }
         prev = t;
       }
       if (ok && prev >= 0) {
@@ -413,7 +415,8 @@ cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, const __half* D, int n, in
   const double products = first + 3.0 * iters + 2.0 * last_y;
   const double flops = 3.0 * 2.0 * kN * kN * static_cast<double>(kN) * products * static_cast<double>(n);
   const int slot = prof_begin(kProfNdbFused, stream, flops);
-  ndb_fused_kernel<<<grid, kThreads, kSmemBytes, stream>>>(my, mz, md, n, alpha_d, plan, status);
+  const int skip = take_load_fault() ? 1 : 0;
+  ndb_fused_kernel<<<grid, kThreads, kSmemBytes, stream>>>(my, mz, md, n, alpha_d, plan, skip, status);
   prof_end(slot, stream);
   prof_count_launch();
   return cudaGetLastError();

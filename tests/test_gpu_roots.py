@@ -142,9 +142,10 @@ def test_standalone_workload_full_size(torch):
 
 @pytest.mark.parametrize("B", [128, 256])
 def test_bounded_wait_reports_timeout_and_context_survives(torch, B):
-    # a GEMM launch that never receives its operand tiles: every wait gives up
+    # a product kernel that never receives its operands: every wait gives up
     # after its limit, the status word says TIMEOUT, and the next call works
-    # (B=128: 128 x 128 tiles; B=256: 128 x 256 tiles)
+    # (B=128: Newton-DB on resident factors, the call's first product kernel;
+    # B=256: the GEMM with 128 x 256 tiles)
     from matrix_inverse_roots_stack_b200 import binding as bd
     A = workloads.spd_stack_geometric(1, B, 10.0, seed=12)
     lib = bd.load()

@@ -202,3 +202,17 @@ def test_get_status_before_any_step(lib):
     assert lib.shampoo_get_status(ctx, ctypes.byref(flags)) == bd.SHAMPOO_OK and flags.value == 0
     assert lib.shampoo_get_status(None, ctypes.byref(flags)) == bd.SHAMPOO_EINVAL
     lib.shampoo_destroy(ctx)
+
+
+def test_profile_read_size(lib):
+    # eight timed stages of (ms, count, flops) and three counters: the header,
+    # the library and the binding agree on 27 values
+    n = 3 * len(bd.PROFILE_STAGES) + 3
+    assert n == 27
+    text = " ".join(open(os.path.join(HEADER_DIR, "dash_b200.h")).read().split()).replace(" * ", " ")
+    assert f"out[0 .. {n - 1}]" in text and f"n >= {n}." in text
+    buf = (ctypes.c_double * n)()
+    assert lib.shampoo_profile_read(buf, n - 1) == bd.SHAMPOO_EINVAL
+    assert lib.shampoo_profile_reset() == 0
+    assert lib.shampoo_profile_read(buf, n) == 0
+    assert list(buf)[:3 * len(bd.PROFILE_STAGES)] == [0.0] * (3 * len(bd.PROFILE_STAGES))

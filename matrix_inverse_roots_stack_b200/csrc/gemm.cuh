@@ -94,7 +94,9 @@ cudaError_t launch_gemm_split(const OpBuffers* bufs, const GemmArgs& args, cudaS
 // OpBuffers), in this order: if first, Y <- Y + Y D with D read from the
 // split stack D; `iters` times D = alpha_d Zhat Y + I/2, Y <- Y + Y D,
 // Zhat <- Zhat + D Zhat; if last_y, once more D = alpha_d Zhat Y + I/2,
-// Y <- Y + Y D (Zhat is then left as it was).  The products' arithmetic is
+// Y <- Y + Y D.  Zhat is written back only when the launch ends with a full
+// iteration (with last_y, or first alone, the Zhat stack keeps what it held
+// before the launch).  The products' arithmetic is
 // that of launch_gemm_split.  Returns cudaErrorNotSupported unless B == 128
 // and first, last_y are 0 or 1.
 cudaError_t launch_ndb_fused(__half* Y, __half* Zhat, const __half* D, int n, int B, float alpha_d, int first,

@@ -81,7 +81,7 @@ constexpr int kBarsOff = 3 * kMatBytes;
 //   iters   full iterations: D = alpha_d Zhat Y + I/2, Y <- Y + Y D,
 //           Zhat <- Zhat + D Zhat;
 //   last_y  one more iteration that updates Y only (the last of a stage
-//           whose Zhat is not used afterwards).
+//           whose Zhat is not used afterwards; Zhat is then not stored).
 struct FusedPlan {
   int first, iters, last_y;
 };
@@ -201,8 +201,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = bars->tmem_slot;
   const int groups = plan_groups(plan);
-  // Zhat changes only in full iterations, and is stored back when the last
-  // group is one
+  // Zhat is stored back only when the last group is a full iteration: after
+  // a last_y group the caller has no further use for it (and after first
+  // alone it is unchanged)
   const bool store_z = group_kind(plan, groups - 1) == kFull;
 
   if (warp == 0) {
